@@ -1,0 +1,248 @@
+// Plain, slow, single-threaded CPU oracle for the 8-bit group-affine
+// quantized linear layer ("MlxInt8Weight" API page).
+//
+// TEST INFRASTRUCTURE ONLY. This file is the independent checker of the CUDA
+// library. Only the test suite, the smoke check and the CPU-baseline leg of the
+// benchmark may load it. It shares no code, header, table or helper with the
+// CUDA path under weight_only_quantized_mlx_b200/csrc, and it includes nothing
+// from there.
+//
+// Build: g++ -O2 -ffp-contract=off -shared -fPIC (see oracle/build.py).
+// -ffp-contract=off keeps every multiply and add a separately rounded
+// operation unless std::fma is written explicitly.
+//
+// What each function follows (MlxInt8Weight page):
+//   * struct fields "packed", "scales", "biases": packed is
+//     [out_features, in_features/4] bytes held in uint32 words; scales and
+//     biases are [out_features, in_features/group_size] BF16, one per group.
+//   * "load": group_size must divide in_features.
+//   * "dequantize_to": the full dequantised weight, BF16.
+//   * "gemv": y = W x.
+//   * "gemv_silu_gate": y = W (silu(gate) * up).
+//   * "gemv_silu_gate_resid": y[n] = x_resid[n] + sum_k W[n,k]*(silu(gate[k])*up[k]).
+//   * "gemm": Y = X W^T, X [m, in_features], Y [m, out_features].
+//
+// Readings taken where the page is silent (each is listed in the design doc):
+//   * q[n,k] is byte (k mod 4) of word packed[n, k/4], little-endian
+//     (byte j = bits 8j..8j+7), unsigned 0..255.
+//   * W[n,k] = bf16_rne( fma_f32(s[n,g], q[n,k], b[n,g]) ), g = floor(k/gs):
+//     groups are gs consecutive columns of one row.
+//   * Products accumulate in fp64 in the order k = 0..K-1 over the BF16 W.
+//   * silu(t) = t / (1 + exp(-t)), in fp64; silu(gate)*up is NOT rounded.
+//   * Each output is rounded once, fp64 -> BF16, round to nearest even.
+//
+// Parity status of every function: pinned (see tests/test_oracle.py).
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+namespace {
+
+// ---- BF16 (1 sign, 8 exponent, 7 stored significand bits) -----------------
+
+// fp32 -> bf16, round to nearest, ties to even, written on the bit pattern.
+// NaN stays NaN (quiet bit forced); infinities and overflow behave as IEEE.
+uint16_t f32_to_bf16(float v) {
+    uint32_t u;
+    std::memcpy(&u, &v, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu) != 0u) {
+        return static_cast<uint16_t>((u >> 16) | 0x0040u);  // quiet NaN
+    }
+    const uint32_t lsb = (u >> 16) & 1u;       // last kept bit
+    const uint32_t rounded = u + 0x7FFFu + lsb;  // half-way goes to even
+    return static_cast<uint16_t>(rounded >> 16);
+}
+
+// fp64 -> bf16 with ONE rounding (nearest, ties to even). Written from the
+// format's definition: a bf16 number is an integer multiple of its quantum
+// 2^(e-8) where 2^(e-1) <= |v| < 2^e, the quantum never going below the
+// subnormal step 2^-133; magnitudes that round to 2^128 or above overflow.
+uint16_t f64_to_bf16(double v) {
+    if (std::isnan(v)) return 0x7FC0u;
+    if (v == 0.0) return std::signbit(v) ? 0x8000u : 0x0000u;
+    if (std::isinf(v)) return v > 0 ? 0x7F80u : 0xFF80u;
+    int e = 0;
+    std::frexp(v, &e);                       // |v| = m * 2^e, 0.5 <= m < 1
+    const int qexp = (e < -125 ? -125 : e) - 8;  // quantum 2^qexp
+    double r = std::nearbyint(std::ldexp(v, -qexp));  // ties to even (default mode)
+    r = std::ldexp(r, qexp);
+    if (std::fabs(r) >= std::ldexp(1.0, 128)) return v > 0 ? 0x7F80u : 0xFF80u;
+    const float f = static_cast<float>(r);  // exact: r has <= 8 significant bits
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    return static_cast<uint16_t>(u >> 16);
+}
+
+float bf16_to_f32(uint16_t h) {
+    const uint32_t u = static_cast<uint32_t>(h) << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    return f;
+}
+
+// ---- the weight encoding ----------------------------------------------------
+
+// Code q[n,k]: byte (k mod 4) of word packed[n, k/4], little-endian.
+inline uint32_t code_at(const uint32_t* packed, int64_t K, int64_t n, int64_t k) {
+    const uint32_t word = packed[n * (K / 4) + k / 4];
+    return (word >> (8 * (k % 4))) & 0xFFu;
+}
+
+// fp32 value of the affine map before rounding: fma(s, q, b).
+inline float affine_f32(const uint32_t* packed, const uint16_t* scales,
+                        const uint16_t* biases, int64_t K, int64_t gs,
+                        int64_t n, int64_t k) {
+    const int64_t G = K / gs;
+    const int64_t g = k / gs;
+    const float s = bf16_to_f32(scales[n * G + g]);
+    const float b = bf16_to_f32(biases[n * G + g]);
+    const float q = static_cast<float>(code_at(packed, K, n, k));
+    return std::fma(s, q, b);
+}
+
+// Row n of the BF16 weight, widened to double (exact).
+void weight_row_f64(const uint32_t* packed, const uint16_t* scales,
+                    const uint16_t* biases, int64_t K, int64_t gs, int64_t n,
+                    double* row) {
+    for (int64_t k = 0; k < K; ++k) {
+        const uint16_t w = f32_to_bf16(affine_f32(packed, scales, biases, K, gs, n, k));
+        row[k] = static_cast<double>(bf16_to_f32(w));
+    }
+}
+
+double silu_f64(double t) { return t / (1.0 + std::exp(-t)); }
+
+}  // namespace
+
+extern "C" {
+
+// ---- scalar conversions (exposed so the tests can pin them) ---------------
+uint16_t oracle_bf16_from_f32(float v) { return f32_to_bf16(v); }
+uint16_t oracle_bf16_from_f64(double v) { return f64_to_bf16(v); }
+float oracle_f32_from_bf16(uint16_t h) { return bf16_to_f32(h); }
+double oracle_silu(double t) { return silu_f64(t); }
+
+// ---- unpack: q[n,k] for the whole [N, K] weight ---------------------------
+void oracle_unpack(const uint32_t* packed, int64_t N, int64_t K, uint8_t* q) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            q[n * K + k] = static_cast<uint8_t>(code_at(packed, K, n, k));
+}
+
+// ---- dequantize_to ----------------------------------------------------------
+// fp32 affine values before the BF16 rounding.
+void oracle_dequant_f32(const uint32_t* packed, const uint16_t* scales,
+                        const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                        float* w) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            w[n * K + k] = affine_f32(packed, scales, biases, K, gs, n, k);
+}
+
+// The BF16 weight, row-major [N, K], as bit patterns.
+void oracle_dequant(const uint32_t* packed, const uint16_t* scales,
+                    const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                    uint16_t* w) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            w[n * K + k] = f32_to_bf16(affine_f32(packed, scales, biases, K, gs, n, k));
+}
+
+// ---- gemv: y = W x ------------------------------------------------------------
+void oracle_gemv_f64(const uint32_t* packed, const uint16_t* scales,
+                     const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                     const uint16_t* x, double* y) {
+    std::vector<double> row(static_cast<size_t>(K));
+    for (int64_t n = 0; n < N; ++n) {
+        weight_row_f64(packed, scales, biases, K, gs, n, row.data());
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) acc += row[k] * static_cast<double>(bf16_to_f32(x[k]));
+        y[n] = acc;
+    }
+}
+
+void oracle_gemv(const uint32_t* packed, const uint16_t* scales,
+                 const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                 const uint16_t* x, uint16_t* y) {
+    std::vector<double> acc(static_cast<size_t>(N));
+    oracle_gemv_f64(packed, scales, biases, N, K, gs, x, acc.data());
+    for (int64_t n = 0; n < N; ++n) y[n] = f64_to_bf16(acc[n]);
+}
+
+// ---- silu gate: h[k] = silu(gate[k]) * up[k] (fp64, never rounded) ---------
+void oracle_silu_gate_f64(const uint32_t* packed, const uint16_t* scales,
+                          const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                          const uint16_t* gate, const uint16_t* up, double* y) {
+    std::vector<double> h(static_cast<size_t>(K));
+    for (int64_t k = 0; k < K; ++k)
+        h[k] = silu_f64(bf16_to_f32(gate[k])) * static_cast<double>(bf16_to_f32(up[k]));
+    std::vector<double> row(static_cast<size_t>(K));
+    for (int64_t n = 0; n < N; ++n) {
+        weight_row_f64(packed, scales, biases, K, gs, n, row.data());
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) acc += row[k] * h[k];
+        y[n] = acc;
+    }
+}
+
+void oracle_silu_gate(const uint32_t* packed, const uint16_t* scales,
+                      const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                      const uint16_t* gate, const uint16_t* up, uint16_t* y) {
+    std::vector<double> acc(static_cast<size_t>(N));
+    oracle_silu_gate_f64(packed, scales, biases, N, K, gs, gate, up, acc.data());
+    for (int64_t n = 0; n < N; ++n) y[n] = f64_to_bf16(acc[n]);
+}
+
+// ---- silu gate + residual: y[n] = x_resid[n] + sum_k W[n,k] h[k] -------------
+void oracle_silu_gate_resid_f64(const uint32_t* packed, const uint16_t* scales,
+                                const uint16_t* biases, int64_t N, int64_t K,
+                                int64_t gs, const uint16_t* gate, const uint16_t* up,
+                                const uint16_t* x_resid, double* y) {
+    oracle_silu_gate_f64(packed, scales, biases, N, K, gs, gate, up, y);
+    for (int64_t n = 0; n < N; ++n) y[n] = static_cast<double>(bf16_to_f32(x_resid[n])) + y[n];
+}
+
+void oracle_silu_gate_resid(const uint32_t* packed, const uint16_t* scales,
+                            const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                            const uint16_t* gate, const uint16_t* up,
+                            const uint16_t* x_resid, uint16_t* y) {
+    std::vector<double> acc(static_cast<size_t>(N));
+    oracle_silu_gate_resid_f64(packed, scales, biases, N, K, gs, gate, up, x_resid, acc.data());
+    for (int64_t n = 0; n < N; ++n) y[n] = f64_to_bf16(acc[n]);
+}
+
+// BF16-materialised silu(gate)*up, for the unfused-chain comparison.
+void oracle_silu_mul(const uint16_t* gate, const uint16_t* up, int64_t K, uint16_t* h) {
+    for (int64_t k = 0; k < K; ++k)
+        h[k] = f64_to_bf16(silu_f64(bf16_to_f32(gate[k])) * static_cast<double>(bf16_to_f32(up[k])));
+}
+
+// ---- gemm: Y[i,n] = sum_k X[i,k] W[n,k], X [m, K], Y [m, N] ----------------
+void oracle_gemm_f64(const uint32_t* packed, const uint16_t* scales,
+                     const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                     const uint16_t* X, int64_t m, double* Y) {
+    std::vector<double> xd(static_cast<size_t>(m * K));
+    for (int64_t t = 0; t < m * K; ++t) xd[t] = static_cast<double>(bf16_to_f32(X[t]));
+    std::vector<double> row(static_cast<size_t>(K));
+    for (int64_t n = 0; n < N; ++n) {
+        weight_row_f64(packed, scales, biases, K, gs, n, row.data());
+        for (int64_t i = 0; i < m; ++i) {
+            const double* xi = xd.data() + i * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += xi[k] * row[k];
+            Y[i * N + n] = acc;
+        }
+    }
+}
+
+void oracle_gemm(const uint32_t* packed, const uint16_t* scales,
+                 const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                 const uint16_t* X, int64_t m, uint16_t* Y) {
+    std::vector<double> acc(static_cast<size_t>(m * N));
+    oracle_gemm_f64(packed, scales, biases, N, K, gs, X, m, acc.data());
+    for (int64_t t = 0; t < m * N; ++t) Y[t] = f64_to_bf16(acc[t]);
+}
+
+}  // extern "C"
