@@ -1,0 +1,166 @@
+/*
+ * mlxq.h - C ABI of the B200 (sm_100a) library for the 8-bit group-affine
+ * quantized linear layer described on the "MlxInt8Weight" API page.
+ *
+ * The weight format (page: struct MlxInt8Weight, fields packed/scales/biases):
+ *   packed  uint32 [out_features, in_features/4], row-major.  Each word holds
+ *           four unsigned 8-bit codes; byte j (bits 8j..8j+7) of word w of a
+ *           row is the code of column 4w+j (little-endian).
+ *   scales  BF16 [out_features, in_features/group_size], row-major.
+ *   biases  BF16 [out_features, in_features/group_size], row-major.
+ *   Weight element: W[n,k] = bf16( fma_f32(scale[n,g], q[n,k], bias[n,g]) ),
+ *   g = k / group_size (groups are group_size consecutive columns of a row).
+ *
+ * Conventions for every call:
+ *   - Device pointers are plain CUDA device addresses.  BF16 buffers hold
+ *     IEEE bfloat16 values (2 bytes each), contiguous, row-major.
+ *   - `stream` is a cudaStream_t value cast to uint64_t (0 = legacy default
+ *     stream).  Kernel calls are asynchronous on that stream; inputs must stay
+ *     valid and outputs untouched by others until the stream passes the call.
+ *   - Every call returns MLXQ_OK (0) or one of the MLXQ_ERR_* codes below and
+ *     launches nothing when it fails validation.  mlxq_last_error() gives a
+ *     human-readable message for the last failure on the calling thread.
+ *   - Accumulation is fp32 on the GPU; each output element is rounded once to
+ *     BF16 (round to nearest even).
+ *   - Outputs may not overlap inputs, except y == x_resid exactly (each
+ *     output element reads its own residual before its single write).  Other
+ *     overlaps that the library can see are rejected with MLXQ_ERR_INVALID_ARG.
+ *   - The calls allocate no device memory per call.
+ */
+#ifndef MLXQ_H
+#define MLXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLXQ_API __attribute__((visibility("default")))
+#else
+#define MLXQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    MLXQ_OK = 0,
+    MLXQ_ERR_INVALID_ARG = 1,    /* null/released handle, null or misaligned pointer, overlap */
+    MLXQ_ERR_PARSE = 2,          /* malformed safetensors blob */
+    MLXQ_ERR_MISSING_TENSOR = 3, /* {base}.weight / .scales / .biases absent */
+    MLXQ_ERR_DTYPE = 4,          /* weight not U32, or scales/biases not BF16 */
+    MLXQ_ERR_SHAPE = 5,          /* weight not 2-D, or scales/biases not [N, K/gs] */
+    MLXQ_ERR_GROUP_SIZE = 6,     /* group_size == 0 or group_size does not divide in_features */
+    MLXQ_ERR_UNSUPPORTED = 7,    /* valid request outside what the kernels handle */
+    MLXQ_ERR_CUDA = 8,           /* CUDA allocation, copy or launch error */
+    MLXQ_ERR_DEVICE_TIMEOUT = 9  /* a kernel gave up a bounded wait (see mlxq_device_status) */
+};
+
+/*
+ * One quantized linear weight resident on the GPU (page: struct
+ * MlxInt8Weight).  N = out_features, K = in_features, gs = group_size.
+ * A handle filled by mlxq_load owns its three buffers and must be freed once
+ * with mlxq_release.  A caller may instead fill the struct with device
+ * buffers it owns (same layouts); such a handle must not be passed to
+ * mlxq_release.
+ */
+typedef struct mlxq_weight {
+    void* packed;          /* uint32 [N, K/4] */
+    void* scales;          /* bf16  [N, K/gs] */
+    void* biases;          /* bf16  [N, K/gs] */
+    uint32_t out_features; /* N */
+    uint32_t in_features;  /* K (a multiple of 4) */
+    uint32_t group_size;   /* gs, divides K */
+} mlxq_weight;
+
+/*
+ * mlxq_load (page: MlxInt8Weight::load).  Parses an in-memory safetensors
+ * blob (host memory, `blob_len` bytes: u64 little-endian header length, JSON
+ * header, data), finds "{base}.weight" (U32, 2-D [N, K/4]), "{base}.scales"
+ * and "{base}.biases" (BF16, [N, K/gs]), allocates three device buffers with
+ * cudaMalloc on the current device and copies the tensors in (synchronous).
+ * On success *out owns the buffers.  Fails, allocating nothing, with
+ * MLXQ_ERR_PARSE, _MISSING_TENSOR, _DTYPE, _SHAPE or _GROUP_SIZE exactly as
+ * the page lists; MLXQ_ERR_CUDA if allocation or the copy fails (partial
+ * allocations are freed).  *out is zeroed on failure.
+ */
+MLXQ_API int mlxq_load(const void* blob, size_t blob_len, const char* base, uint32_t group_size,
+              mlxq_weight* out);
+
+/*
+ * mlxq_dequant (page: MlxInt8Weight::dequantize_to, kernel mlx_int8_dequant).
+ * Writes the full dequantised weight as BF16 to `out`, row-major [N, K]:
+ * out must hold at least N*K*2 bytes (device).  Bytes past N*K*2 are not
+ * touched.  Bit-exact: each element is bf16_rne(fma_f32(s, q, b)).
+ */
+MLXQ_API int mlxq_dequant(const mlxq_weight* w, void* out, uint64_t stream);
+
+/*
+ * mlxq_gemv (page: MlxInt8Weight::gemv, kernel mlx_int8_gemv).
+ * y = W x.  x: BF16 [K] (device); y: BF16, at least N elements (device).
+ */
+MLXQ_API int mlxq_gemv(const mlxq_weight* w, const void* x, void* y, uint64_t stream);
+
+/*
+ * mlxq_gemv_silu_gate (page: MlxInt8Weight::gemv_silu_gate, kernel
+ * mlx_int8_gemv_silu_gate).  y = W (silu(gate) * up), silu(t) = t/(1+e^-t),
+ * in one launch; silu(gate)*up is formed in registers and never written to
+ * memory.  gate, up: BF16 [K]; y: BF16 [N].
+ */
+MLXQ_API int mlxq_gemv_silu_gate(const mlxq_weight* w, const void* gate, const void* up, void* y,
+                        uint64_t stream);
+
+/*
+ * mlxq_gemv_silu_gate_resid (page: MlxInt8Weight::gemv_silu_gate_resid).
+ * y[n] = x_resid[n] + sum_k W[n,k] * (silu(gate[k]) * up[k]), one launch.
+ * gate, up: BF16 [K]; x_resid, y: BF16 [N].  y may equal x_resid exactly.
+ */
+MLXQ_API int mlxq_gemv_silu_gate_resid(const mlxq_weight* w, const void* gate, const void* up,
+                              const void* x_resid, void* y, uint64_t stream);
+
+/*
+ * mlxq_gemm (page: MlxInt8Weight::gemm, kernel mlx_int8_gemm).
+ * Y = X W^T.  X: BF16 [m, K] row-major; Y: BF16 [m, N] row-major.  m == 0 is
+ * a no-op.  The kernel is chosen from m: the m == 1 stream kernel, a CUDA-core
+ * small-m kernel, or the tcgen05 tensor-core kernel (weight tiles
+ * dequantised to BF16 in shared memory, fp32 accumulators in TMEM).
+ */
+MLXQ_API int mlxq_gemm(const mlxq_weight* w, const void* x, void* y, uint32_t m, uint64_t stream);
+
+/* Kernel selection for mlxq_gemm_with (tests and benchmarks pin a path). */
+enum {
+    MLXQ_GEMM_AUTO = 0,    /* what mlxq_gemm picks */
+    MLXQ_GEMM_ROWS = 1,    /* m independent passes of the gemv stream kernel */
+    MLXQ_GEMM_SMALLM = 2,  /* CUDA-core small-m kernel (m <= 32) */
+    MLXQ_GEMM_TCGEN05 = 3  /* tensor-core kernel */
+};
+
+/* mlxq_gemm with an explicit kernel; MLXQ_ERR_UNSUPPORTED if that kernel
+ * cannot take this shape. */
+MLXQ_API int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kernel,
+                   uint64_t stream);
+
+/*
+ * mlxq_release (page: MlxInt8Weight::release).  Frees the three buffers of a
+ * handle filled by mlxq_load and zeroes the handle.  The buffers are freed
+ * exactly once: a second call on the same handle returns MLXQ_ERR_INVALID_ARG.
+ */
+MLXQ_API int mlxq_release(mlxq_weight* w);
+
+/* Message for the last nonzero status returned on this thread ("" if none). */
+MLXQ_API const char* mlxq_last_error(void);
+
+/*
+ * Waits for the current device to go idle, then reads and clears the
+ * library's device status word.  Returns MLXQ_OK, or MLXQ_ERR_DEVICE_TIMEOUT
+ * if some kernel since the last check gave up a bounded wait (its outputs are
+ * then not valid), or MLXQ_ERR_CUDA.  Kernels never hang or trap on a stalled
+ * pipeline: they record the timeout here and return.
+ */
+MLXQ_API int mlxq_device_status(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLXQ_H */

@@ -1,0 +1,324 @@
+"""GPU parity: every kernel of the library, called through the C ABI, against
+the CPU oracle on the same seeded inputs.
+
+* dequantize_to: bit-exact (BF16 bit patterns equal).
+* gemv / gemv_silu_gate / gemv_silu_gate_resid / gemm: within the tolerance
+  in tests/_helpers.py, elementwise and normwise.
+Sizes span several pipeline stages / tiles with ragged tails, both the
+vectorised and the generic kernel paths, and the workload shapes of the API
+page's use (decode projections, a fused MLP, small-m and prefill gemm); at the
+largest shapes the oracle is evaluated on sampled weight rows.  Output buffers
+carry sentinel guard bands that must survive every call.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_only_quantized_mlx_b200 as mq
+from _helpers import Guarded, assert_close, dev, host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    mq.lib()
+    yield
+    torch.cuda.synchronize()
+    mq.mlxq_device_status()  # no kernel gave up a bounded wait
+
+
+class DevWeight:
+    def __init__(self, packed, scales, biases, gs):
+        self.host = (packed, scales, biases)
+        self.t = (dev(packed), dev(scales), dev(biases))
+        self.gs = gs
+        self.w = mq.weight_view(*self.t, gs)
+        self.N, self.K = packed.shape[0], packed.shape[1] * 4
+
+
+def make(seed, N, K, gs):
+    g = synth.rng(seed)
+    p, s, b = synth.weight(g, N, K, gs)
+    return DevWeight(p, s, b, gs), g
+
+
+def rows_subset(W: DevWeight, rows):
+    p, s, b = W.host
+    return p[rows], s[rows], b[rows]
+
+
+# ---------------------------------------------------------------- dequantize_to
+DEQ_SHAPES = [
+    (256, 512, 64),    # the tiny workload
+    (256, 512, 32), (256, 512, 128), (37, 1040, 16), (3, 64, 64), (1, 16, 16),
+    (5, 12, 4), (9, 60, 12), (4, 8, 2), (6, 20, 20), (2, 4, 1),   # generic path
+]
+
+
+@pytest.mark.parametrize("N,K,gs", DEQ_SHAPES)
+def test_dequant_bit_exact(N, K, gs):
+    W, _ = make(0, N, K, gs)
+    out = Guarded(N * K)
+    mq.mlxq_dequant(W.w, out.data_ptr())
+    torch.cuda.synchronize()
+    out.check_guards()
+    ref = oracle.dequant(*W.host, gs)
+    assert np.array_equal(out.value_bits(), ref.ravel())
+
+
+def test_dequant_misaligned_output_takes_generic_path():
+    W, _ = make(1, 33, 256, 32)
+    out = Guarded(33 * 256, offset_elems=1)  # 2-byte but not 16-byte aligned
+    mq.mlxq_dequant(W.w, out.data_ptr())
+    torch.cuda.synchronize()
+    out.check_guards()
+    assert np.array_equal(out.value_bits(), oracle.dequant(*W.host, 32).ravel())
+
+
+def test_dequant_decode_workload_100_pairs():
+    out = torch.empty(4096 * 4096, dtype=torch.bfloat16, device="cuda")
+    for seed in range(100):
+        p, s, b, _ = synth.decode_pair(seed, 4096, 4096, 64)
+        W = DevWeight(p, s, b, 64)
+        mq.mlxq_dequant(W.w, out)
+        got = host_bits(out)
+        ref = oracle.dequant(p, s, b, 64).ravel()
+        assert np.array_equal(got, ref), f"seed {seed}"
+
+
+def test_dequant_loaded_weight_and_release():
+    g = synth.rng(5)
+    p, s, b = synth.weight(g, 64, 256, 64)
+    W = mq.MlxInt8Weight.load(synth.weight_blob("model.layers.0.mlp.down_proj", p, s, b),
+                              "model.layers.0.mlp.down_proj", 64)
+    assert (W.out_features, W.in_features, W.group_size) == (64, 256, 64)
+    out = torch.empty(64 * 256, dtype=torch.bfloat16, device="cuda")
+    W.dequantize_to(out)
+    assert np.array_equal(host_bits(out), oracle.dequant(p, s, b, 64).ravel())
+    W.release()
+    with pytest.raises(mq.MlxqError):
+        W.release()
+
+
+# ---------------------------------------------------------------- gemv
+GEMV_SHAPES = [
+    (256, 512, 64),                     # tiny workload
+    (4096, 4096, 64), (4096, 4096, 128), (4096, 4096, 32),
+    (1000, 2048, 64), (333, 1024, 16), (17, 8192, 64),
+    (2048, 14336, 64), (517, 14336, 128), (300, 28672, 64),  # 2 and 4 chunks per thread
+    (129, 256, 32), (7, 64, 64), (1, 16, 16),
+    (45, 36, 12), (10, 100, 4), (3, 40000, 64),              # generic path
+]
+
+
+def run_gemv(W, x_bits):
+    x = dev(x_bits)
+    y = Guarded(W.N)
+    mq.mlxq_gemv(W.w, x, y.data_ptr())
+    torch.cuda.synchronize()
+    y.check_guards()
+    return y.value_bits()
+
+
+@pytest.mark.parametrize("N,K,gs", GEMV_SHAPES)
+def test_gemv(N, K, gs):
+    W, g = make(2, N, K, gs)
+    x = synth.activations(g, K)
+    assert_close(run_gemv(W, x), oracle.gemv(*W.host, gs, x), f"gemv {N}x{K}/{gs}")
+
+
+def test_gemv_decode_workload_100_pairs():
+    for seed in range(100):
+        p, s, b, x = synth.decode_pair(seed, 4096, 4096, 64)
+        W = DevWeight(p, s, b, 64)
+        assert_close(run_gemv(W, x), oracle.gemv(p, s, b, 64, x), f"seed {seed}")
+
+
+def test_gemv_misaligned_x_takes_generic_path():
+    W, g = make(3, 200, 1024, 64)
+    x_bits = synth.activations(g, 1024)
+    buf = torch.empty(1024 + 8, dtype=torch.bfloat16, device="cuda")
+    xs = buf[1:1025]
+    xs.copy_(dev(x_bits))
+    y = Guarded(200)
+    mq.mlxq_gemv(W.w, xs, y.data_ptr())
+    torch.cuda.synchronize()
+    y.check_guards()
+    assert_close(y.value_bits(), oracle.gemv(*W.host, 64, x_bits))
+
+
+def test_gemv_integer_weights_are_exact():
+    # s = 1, b = 0, small-integer x: every fp32 sum is exact, so the GPU must
+    # return exactly the oracle's (exact) result.
+    g = np.random.default_rng(11)
+    N, K = 300, 4096
+    q = g.integers(0, 256, size=(N, K), dtype=np.uint8)
+    packed = q.reshape(N, K // 4, 4).view("<u4").reshape(N, K // 4).astype(np.uint32)
+    s = np.full((N, K // 64), 0x3F80, np.uint16)
+    b = np.zeros((N, K // 64), np.uint16)
+    x = synth.to_bf16_bits(g.integers(-3, 4, size=K).astype(np.float32))
+    W = DevWeight(packed, s, b, 64)
+    got = run_gemv(W, x)
+    assert np.array_equal(got, oracle.gemv(packed, s, b, 64, x))
+
+
+# ---------------------------------------------------------------- silu gate (+ resid)
+SILU_SHAPES = [(4096, 14336, 64), (256, 512, 64), (1000, 4096, 128), (77, 2048, 32),
+               (300, 28672, 64), (45, 36, 12)]
+
+
+@pytest.mark.parametrize("N,K,gs", SILU_SHAPES)
+def test_gemv_silu_gate(N, K, gs):
+    W, g = make(4, N, K, gs)
+    gate, up = synth.activations(g, K), synth.activations(g, K)
+    y = Guarded(N)
+    mq.mlxq_gemv_silu_gate(W.w, dev(gate), dev(up), y.data_ptr())
+    torch.cuda.synchronize()
+    y.check_guards()
+    assert_close(y.value_bits(), oracle.silu_gate(*W.host, gs, gate, up), f"silu {N}x{K}")
+
+
+@pytest.mark.parametrize("N,K,gs", SILU_SHAPES)
+def test_gemv_silu_gate_resid(N, K, gs):
+    W, g = make(5, N, K, gs)
+    gate, up, r = synth.activations(g, K), synth.activations(g, K), synth.activations(g, N)
+    y = Guarded(N)
+    mq.mlxq_gemv_silu_gate_resid(W.w, dev(gate), dev(up), dev(r), y.data_ptr())
+    torch.cuda.synchronize()
+    y.check_guards()
+    assert_close(y.value_bits(), oracle.silu_gate_resid(*W.host, gs, gate, up, r), f"resid {N}x{K}")
+
+
+def test_resid_in_place():
+    W, g = make(6, 1024, 4096, 64)
+    gate, up, r = synth.activations(g, 4096), synth.activations(g, 4096), synth.activations(g, 1024)
+    yr = dev(r)
+    mq.mlxq_gemv_silu_gate_resid(W.w, dev(gate), dev(up), yr, yr)  # y == x_resid
+    assert_close(host_bits(yr), oracle.silu_gate_resid(*W.host, 64, gate, up, r))
+
+
+def test_zero_gate_gives_zero_and_residual():
+    W, g = make(7, 512, 4096, 64)
+    zero = np.zeros(4096, np.uint16)
+    up, r = synth.activations(g, 4096), synth.activations(g, 512)
+    y = torch.empty(512, dtype=torch.bfloat16, device="cuda")
+    mq.mlxq_gemv_silu_gate(W.w, dev(zero), dev(up), y)
+    assert np.all(host_bits(y) & 0x7FFF == 0)  # +-0
+    mq.mlxq_gemv_silu_gate_resid(W.w, dev(zero), dev(up), dev(r), y)
+    assert np.array_equal(host_bits(y), r)
+
+
+def test_fused_mlp_chain():
+    """x -> gate, up projections (N=14336, K=4096) -> silu_gate_resid down
+    projection (N=4096, K=14336).  The down projection is checked against the
+    oracle fed with the GPU's BF16 gate/up, and against the unfused oracle
+    (silu(gate)*up materialised in BF16)."""
+    D, F, gs = 4096, 14336, 64
+    Wg, g = make(30, F, D, gs)
+    Wu, _ = make(31, F, D, gs)
+    Wd, _ = make(32, D, F, gs)
+    x = synth.activations(g, D)
+    xr = synth.activations(g, D)
+    gate = torch.empty(F, dtype=torch.bfloat16, device="cuda")
+    up = torch.empty(F, dtype=torch.bfloat16, device="cuda")
+    xd = dev(x)
+    mq.mlxq_gemv(Wg.w, xd, gate)
+    mq.mlxq_gemv(Wu.w, xd, up)
+    y = torch.empty(D, dtype=torch.bfloat16, device="cuda")
+    mq.mlxq_gemv_silu_gate_resid(Wd.w, gate, up, dev(xr), y)
+    gb, ub = host_bits(gate), host_bits(up)
+    assert_close(gb, oracle.gemv(*Wg.host, gs, x), "gate proj")
+    assert_close(ub, oracle.gemv(*Wu.host, gs, x), "up proj")
+    assert_close(host_bits(y), oracle.silu_gate_resid(*Wd.host, gs, gb, ub, xr), "down (fused)")
+    h = oracle.silu_mul(gb, ub)
+    ref_unfused = oracle.f64_to_bf16_array(oracle.gemv_f64(*Wd.host, gs, h) +
+                                           oracle.bf16_bits_to_f64(xr))
+    assert_close(host_bits(y), ref_unfused, "down (unfused reference)")
+
+
+# ---------------------------------------------------------------- gemm
+def run_gemm(W, X_bits, m, kernel=mq.MLXQ_GEMM_AUTO):
+    X = dev(X_bits)
+    Y = Guarded(m * W.N)
+    mq.mlxq_gemm_with(W.w, X, Y.data_ptr(), m, kernel)
+    torch.cuda.synchronize()
+    Y.check_guards()
+    return Y.value_bits().reshape(m, W.N)
+
+
+SMALLM_SHAPES = [(512, 1024, 64), (300, 4096, 32), (256, 14336, 128), (128, 28672, 64), (77, 512, 16)]
+
+
+@pytest.mark.parametrize("N,K,gs", SMALLM_SHAPES)
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 7, 8, 16, 32])
+def test_gemm_smallm(N, K, gs, m):
+    W, g = make(8, N, K, gs)
+    X = synth.activations(g, m, K)
+    ref = oracle.gemm(*W.host, gs, X)
+    assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_SMALLM), ref, f"smallm m={m} {N}x{K}")
+    assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_AUTO), ref, f"auto m={m} {N}x{K}")
+
+
+@pytest.mark.parametrize("m", [1, 3, 9])
+def test_gemm_rows_path_and_generic_shapes(m):
+    W, g = make(9, 45, 36, 12)  # generic shape: only the row passes take it
+    X = synth.activations(g, m, 36)
+    ref = oracle.gemm(*W.host, 12, X)
+    assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_ROWS), ref)
+    assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_AUTO), ref)
+
+
+def test_gemm_m1_equals_gemv_bitwise():
+    W, g = make(10, 1000, 4096, 64)
+    x = synth.activations(g, 4096)
+    assert np.array_equal(run_gemm(W, x.reshape(1, -1), 1)[0], run_gemv(W, x))
+
+
+@pytest.mark.parametrize("NK", [(28672, 8192), (8192, 28672)])
+@pytest.mark.parametrize("gs", [32, 64, 128])
+def test_gemm_smallm_workload_sampled_rows(NK, gs):
+    """The small-m batched-decode shapes at full size; the oracle checks a
+    sample of 256 weight rows (first, last and random) for every m."""
+    N, K = NK
+    W, g = make(20 + gs, N, K, gs)
+    pick = np.unique(np.concatenate([np.arange(64), np.arange(N - 64, N),
+                                     np.random.default_rng(gs).choice(N, 128, replace=False)]))
+    sub = rows_subset(W, pick)
+    for m in (1, 2, 4, 8, 16, 32):
+        X = synth.activations(g, m, K)
+        got = run_gemm(W, X, m)
+        ref = oracle.gemm(*sub, gs, X)
+        assert_close(got[:, pick], ref, f"{N}x{K}/{gs} m={m}")
+
+
+def test_empty_shapes():
+    """N = 0: nothing is written; K = 0: y = 0 (plus the residual); m = 0: no-op."""
+    e32, e16 = np.zeros((0, 16), np.uint32), np.zeros((0, 2), np.uint16)
+    W0 = mq.MlxInt8Weight.load(synth.weight_blob("e", e32, e16, e16), "e", 32)
+    y = Guarded(8)
+    x = dev(synth.activations(synth.rng(1), 64))
+    mq.mlxq_gemv(W0.handle, x, y.data_ptr())
+    mq.mlxq_dequant(W0.handle, y.data_ptr())
+    mq.mlxq_gemm(W0.handle, x, y.data_ptr(), 0)
+    mq.mlxq_gemm(W0.handle, x, y.data_ptr(), 3)
+    torch.cuda.synchronize()
+    y.check_guards()
+    assert np.all(y.value_bits() == 0x7FC1)
+    W0.release()
+
+    k32, k16 = np.zeros((16, 0), np.uint32), np.zeros((16, 0), np.uint16)
+    Wk = mq.MlxInt8Weight.load(synth.weight_blob("k", k32, k16, k16), "k", 4)
+    assert (Wk.out_features, Wk.in_features) == (16, 0)
+    yk = torch.full((16,), 3.0, dtype=torch.bfloat16, device="cuda")
+    mq.mlxq_gemv(Wk.handle, None, yk)
+    assert np.all(host_bits(yk) & 0x7FFF == 0)
+    r = dev(synth.activations(synth.rng(2), 16))
+    mq.mlxq_gemv_silu_gate_resid(Wk.handle, None, None, r, yk)
+    assert np.array_equal(host_bits(yk), host_bits(r))
+    Wk.release()

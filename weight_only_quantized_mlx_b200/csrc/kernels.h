@@ -1,0 +1,49 @@
+// Host-side launch interface between the C ABI (abi.cu) and the kernels.
+// Every launcher validates nothing: abi.cu has already checked pointers,
+// shapes and alignment.  Each returns the launch status (cudaGetLastError).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mlxq {
+
+struct WeightView {
+    const uint32_t* packed;  // [N, K/4]
+    const uint16_t* scales;  // [N, G] bf16 bits
+    const uint16_t* biases;  // [N, G] bf16 bits
+    int64_t N, K, gs, G;
+};
+
+enum GemvMode { GEMV_PLAIN = 0, GEMV_SILU = 1, GEMV_SILU_RESID = 2 };
+
+// Device properties of the current device (cached per device).
+struct DeviceInfo {
+    int device;
+    int sm_count;
+    int max_smem_optin;
+};
+const DeviceInfo& device_info();
+
+// Address of the library's device status word on the current device.
+unsigned int* device_status_ptr();
+
+// mlx_int8_dequant: out [N, K] bf16.
+cudaError_t launch_dequant(const WeightView& w, void* out, cudaStream_t stream);
+
+// mlx_int8_gemv family (m = 1): y = W h (+ resid), h = x or silu(gate)*up.
+cudaError_t launch_gemv(const WeightView& w, int mode, const void* x, const void* gate,
+                        const void* up, const void* resid, void* y, cudaStream_t stream);
+
+// CUDA-core small-m gemm: Y [m, N] = X [m, K] W^T, 2 <= m <= kSmallMMax.
+constexpr int kSmallMMax = 32;
+bool gemm_smallm_supported(const WeightView& w, int64_t m);
+cudaError_t launch_gemm_smallm(const WeightView& w, const void* X, void* Y, int64_t m,
+                               cudaStream_t stream);
+
+// tcgen05 tensor-core gemm.
+bool gemm_tc_supported(const WeightView& w, int64_t m, const void* X, const void* Y);
+cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t m,
+                           cudaStream_t stream);
+
+}  // namespace mlxq
