@@ -213,14 +213,26 @@ def run_gpu(args):
     xp = [x.data_ptr() for x in xs]
     yp = [y.data_ptr() for y in ys]
 
-    def step():
+    def step_on(sp):
         for i in range(N_PAIRS):
-            L.mlxq_gemv(handles[i], xp[i], yp[i], s_ptr)
+            rc = L.mlxq_gemv(handles[i], xp[i], yp[i], sp)
+            if rc:
+                raise mq.MlxqError(rc, mq.mlxq_last_error())
+
+    # The step's 100 launches are captured once in a CUDA graph and replayed:
+    # the launch-bound loop runs without per-launch host overhead.
+    step_on(s_ptr)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step_on(torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
 
     per_launch = gemv_bytes(D_N, D_K, D_GS)
     rows = {}
     with ClockSampler(dev.index or 0) as clk:
-        ms = time_region(step, args.steps, args.warmup, stream, world)
+        ms = time_region(graph.replay, args.steps, args.warmup, stream, world)
+        ms_eager = time_region(lambda: step_on(s_ptr), args.steps, args.warmup, stream, world)
         # e2e: the public call with host buffers; per step and pair, H2D of x
         # from pinned memory, the gemv, D2H of y, all inside the timed region
         xh = [x.cpu().pin_memory() for x in xs]
@@ -238,6 +250,7 @@ def run_gpu(args):
         if args.rows and world == 1:
             rows = measure_rows(mq, torch, synth, dev, stream, weights, peaks, args)
     mq.mlxq_device_status()
+    del graph
 
     total_bytes = per_launch * N_PAIRS * world
     value = total_bytes / (ms * 1e-3) / 1e9
@@ -266,6 +279,8 @@ def run_gpu(args):
             "l2": "inputs larger than L2 (1.78 GB of weights per rank vs 126 MB L2)",
             "weights": "u8 group-affine, bf16 scale/bias", "activations": "bf16",
             "accumulate": "fp32", "parallelism": f"dp{world} (independent problems)",
+            "launch": "CUDA graph of the step's 100 launches",
+            "eager_gbs": round(total_bytes / (ms_eager * 1e-3) / 1e9, 1),
         },
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -429,6 +444,45 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_case(args):
+    """--case KIND:N:K:GS[:M]: run one kernel `--steps` times on a seeded
+    weight, no timing line (the command the committed ncu summaries use).
+    KIND is dequant, gemv, silu, resid, gemm (auto), smallm, rows or tc."""
+    import torch
+    import synth
+    import weight_only_quantized_mlx_b200 as mq
+    parts = args.case.split(":")
+    kind, N, K, gs = parts[0], int(parts[1]), int(parts[2]), int(parts[3])
+    m = int(parts[4]) if len(parts) > 4 else 1
+    torch.cuda.set_device(0)
+    g = synth.rng(7)
+    w = upload_weight(mq, *synth.weight(g, N, K, gs), gs)
+    dev = torch.device("cuda", 0)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    X = to_dev(synth.activations(g, m, K))
+    gate, up = to_dev(synth.activations(g, K)), to_dev(synth.activations(g, K))
+    r = to_dev(synth.activations(g, N))
+    Y = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(N * K, dtype=torch.bfloat16, device=dev) if kind == "dequant" else None
+    kernel = {"gemm": mq.MLXQ_GEMM_AUTO, "smallm": mq.MLXQ_GEMM_SMALLM, "rows": mq.MLXQ_GEMM_ROWS,
+              "tc": mq.MLXQ_GEMM_TCGEN05}.get(kind)
+    for _ in range(args.steps):
+        if kind == "dequant":
+            mq.mlxq_dequant(w.handle, out)
+        elif kind == "gemv":
+            mq.mlxq_gemv(w.handle, X, Y)
+        elif kind == "silu":
+            mq.mlxq_gemv_silu_gate(w.handle, gate, up, Y)
+        elif kind == "resid":
+            mq.mlxq_gemv_silu_gate_resid(w.handle, gate, up, r, Y)
+        else:
+            mq.mlxq_gemm_with(w.handle, X, Y, m, kernel)
+    torch.cuda.synchronize()
+    mq.mlxq_device_status()
+    w.release()
+    print(f"case {args.case}: {args.steps} launches ok")
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -439,9 +493,12 @@ def main(argv=None):
     ap.add_argument("--no-rows", dest="rows", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--case", default=None, help="KIND:N:K:GS[:M] single-kernel run for profiling")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 warm-up steps, always
-    if args.impl == "reference":
+    if args.case:
+        run_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

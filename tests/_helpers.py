@@ -21,8 +21,11 @@ def bits_to_f64(bits) -> np.ndarray:
     return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def assert_close(y_bits, ref_bits, what=""):
-    """GEMV/GEMM tolerance: elementwise and normwise, against the oracle's BF16 output."""
+def assert_close(y_bits, ref_bits, what="", elementwise=True):
+    """GEMV/GEMM tolerance: elementwise and normwise, against the oracle's BF16
+    output.  elementwise=False keeps only the normwise bound (used where the
+    reference is a different, coarser definition, e.g. an unfused chain that
+    rounds an intermediate the fused kernel keeps in fp32)."""
     y = bits_to_f64(y_bits).ravel()
     r = bits_to_f64(ref_bits).ravel()
     assert y.shape == r.shape
@@ -32,7 +35,7 @@ def assert_close(y_bits, ref_bits, what=""):
     mx = np.abs(r).max()
     bound = ELEM_REL * np.abs(r) + ELEM_ABS_OF_MAX * mx
     err = np.abs(y - r)
-    bad = np.nonzero(err > bound)[0]
+    bad = np.nonzero(err > bound)[0] if elementwise else np.zeros(0, dtype=np.int64)
     assert bad.size == 0, (f"{what}: {bad.size} elements outside tolerance; first at {bad[0]}: "
                            f"got {y[bad[0]]!r} want {r[bad[0]]!r} (bound {bound[bad[0]]:.3g})")
     nr = np.linalg.norm(r)

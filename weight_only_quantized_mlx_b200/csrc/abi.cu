@@ -4,6 +4,7 @@
 // step of the layer runs in the CUDA kernels.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cerrno>
 #include <cstdarg>
 #include <cstdio>
@@ -42,7 +43,7 @@ int ok() { return MLXQ_OK; }
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mu;
 DeviceInfo g_dev[kMaxDevices];
-bool g_dev_ok[kMaxDevices];
+std::atomic<bool> g_dev_ready[kMaxDevices];
 unsigned int* g_status_ptr[kMaxDevices];
 
 // ---- minimal JSON reader for the safetensors header ---------------------------------
@@ -381,30 +382,26 @@ const DeviceInfo& device_info() {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= kMaxDevices) dev = 0;
+    if (g_dev_ready[dev].load(std::memory_order_acquire)) return g_dev[dev];
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (!g_dev_ok[dev]) {
+    if (!g_dev_ready[dev].load(std::memory_order_relaxed)) {
         DeviceInfo di{};
         di.device = dev;
         cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
         cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (di.sm_count <= 0) di.sm_count = 1;
         if (di.max_smem_optin <= 0) di.max_smem_optin = 48 * 1024;
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) == cudaSuccess) g_status_ptr[dev] = static_cast<unsigned int*>(p);
         g_dev[dev] = di;
-        g_dev_ok[dev] = true;
+        g_dev_ready[dev].store(true, std::memory_order_release);
     }
     return g_dev[dev];
 }
 
 unsigned int* device_status_ptr() {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= kMaxDevices) dev = 0;
-    std::lock_guard<std::mutex> lk(g_dev_mu);
-    if (!g_status_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_status_word) == cudaSuccess) g_status_ptr[dev] = static_cast<unsigned int*>(p);
-    }
-    return g_status_ptr[dev];
+    const DeviceInfo& di = device_info();
+    return g_status_ptr[di.device];
 }
 
 }  // namespace mlxq

@@ -249,14 +249,19 @@ __global__ void __launch_bounds__(544, 1) k_gemv_stream(const GemvParams p) {
             if ((lane & 3) == 0) rbuf[(mt * 8 + ((lane >> 2) & 7)) * nwc + warp] = v;
         }
         named_bar_sync(1, T);
-        if (tid < 8 * MT && (tid & 7) < rows_g) {
-            const int mt = tid >> 3, r = tid & 7;
-            float acc = 0.f;
-            for (int w = 0; w < nwc; ++w) acc += rbuf[(mt * 8 + r) * nwc + w];
-            const int64_t row = g0 + r;
-            if (MODE == GEMV_SILU_RESID) acc += bf16_bits_to_f32(p.resid[row]);
-            const __nv_bfloat16 o = __float2bfloat16_rn(acc);
-            p.y[static_cast<int64_t>(p.i0 + mt) * p.N + row] = *reinterpret_cast<const uint16_t*>(&o);
+        // warp w finishes outputs w, w + nwc, ...: one partial per lane, then
+        // a fixed shuffle tree (deterministic order)
+        for (int o = warp; o < 8 * MT; o += nwc) {
+            const int mt = o >> 3, r = o & 7;
+            float acc = lane < nwc ? rbuf[(mt * 8 + r) * nwc + lane] : 0.f;
+#pragma unroll
+            for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, sh);
+            if (lane == 0 && r < rows_g) {
+                const int64_t row = g0 + r;
+                if (MODE == GEMV_SILU_RESID) acc += bf16_bits_to_f32(p.resid[row]);
+                const __nv_bfloat16 ob = __float2bfloat16_rn(acc);
+                p.y[static_cast<int64_t>(p.i0 + mt) * p.N + row] = *reinterpret_cast<const uint16_t*>(&ob);
+            }
         }
     }
 }
@@ -306,8 +311,8 @@ inline bool a16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) =
 template <int MODE, int CPT, int B, int MT>
 cudaError_t launch_stream_t(const GemvParams& p, int grid, size_t smem, cudaStream_t stream) {
     auto kern = k_gemv_stream<MODE, CPT, B, MT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    static std::atomic<int> configured[64];
+    cudaError_t e = ensure_dynamic_smem(kern, smem, configured);
     if (e != cudaSuccess) return e;
     kern<<<grid, p.T + 32, smem, stream>>>(p);
     return cudaGetLastError();

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace mlxq {
 
 struct WeightView {
@@ -27,6 +29,24 @@ const DeviceInfo& device_info();
 
 // Address of the library's device status word on the current device.
 unsigned int* device_status_ptr();
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` once per device
+// (cudaFuncSetAttribute is a host round trip; launches then skip it).
+// `configured` is the calling launch site's own per-device record (one static
+// array per kernel instance: kernels of one signature share a function type).
+template <typename Kernel>
+cudaError_t ensure_dynamic_smem(Kernel kern, size_t bytes, std::atomic<int> (&configured)[64]) {
+    const int dev = device_info().device;
+    const int want = static_cast<int>(bytes);
+    if (configured[dev].load(std::memory_order_relaxed) >= want) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, want);
+    if (e == cudaSuccess) {
+        int cur = configured[dev].load(std::memory_order_relaxed);
+        while (cur < want && !configured[dev].compare_exchange_weak(cur, want)) {
+        }
+    }
+    return e;
+}
 
 // mlx_int8_dequant: out [N, K] bf16.
 cudaError_t launch_dequant(const WeightView& w, void* out, cudaStream_t stream);
