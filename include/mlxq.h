@@ -121,18 +121,21 @@ MLXQ_API int mlxq_gemv_silu_gate_resid(const mlxq_weight* w, const void* gate, c
 /*
  * mlxq_gemm (page: MlxInt8Weight::gemm, kernel mlx_int8_gemm).
  * Y = X W^T.  X: BF16 [m, K] row-major; Y: BF16 [m, N] row-major.  m == 0 is
- * a no-op.  The kernel is chosen from m: the m == 1 stream kernel, a CUDA-core
- * small-m kernel, or the tcgen05 tensor-core kernel (weight tiles
- * dequantised to BF16 in shared memory, fp32 accumulators in TMEM).
+ * a no-op.  The kernel is chosen from m: weight-streaming kernels for small m
+ * (every weight byte read once, dequantised in registers) or the tcgen05
+ * tensor-core kernel for larger m (weight tiles dequantised to BF16 in shared
+ * memory, fp32 accumulators in TMEM).
  */
 MLXQ_API int mlxq_gemm(const mlxq_weight* w, const void* x, void* y, uint32_t m, uint64_t stream);
 
 /* Kernel selection for mlxq_gemm_with (tests and benchmarks pin a path). */
 enum {
-    MLXQ_GEMM_AUTO = 0,    /* what mlxq_gemm picks */
-    MLXQ_GEMM_ROWS = 1,    /* m independent passes of the gemv stream kernel */
-    MLXQ_GEMM_SMALLM = 2,  /* CUDA-core small-m kernel (m <= 32) */
-    MLXQ_GEMM_TCGEN05 = 3  /* tensor-core kernel */
+    MLXQ_GEMM_AUTO = 0,        /* what mlxq_gemm picks */
+    MLXQ_GEMM_ROWS = 1,        /* m independent passes of the gemv kernel */
+    MLXQ_GEMM_SMALLM = 2,      /* weight-streaming kernel, products on the tensor pipe
+                                  (mma.sync fragments), m <= 8 */
+    MLXQ_GEMM_TCGEN05 = 3,     /* tcgen05 tensor-core kernel (TMEM accumulators) */
+    MLXQ_GEMM_SMALLM_FFMA = 4  /* weight-streaming kernel on the fp32 pipes, m <= 32 */
 };
 
 /* mlxq_gemm with an explicit kernel; MLXQ_ERR_UNSUPPORTED if that kernel

@@ -114,6 +114,7 @@ GEMV_SHAPES = [
     (2048, 14336, 64), (517, 14336, 128), (300, 28672, 64),  # 2 and 4 chunks per thread
     (129, 256, 32), (7, 64, 64), (1, 16, 16),
     (45, 36, 12), (10, 100, 4), (3, 40000, 64),              # generic path
+    (700, 4096, 256), (90, 8192, 256),                        # fp32-pipe stream kernel
 ]
 
 
@@ -170,7 +171,8 @@ def test_gemv_integer_weights_are_exact():
 
 # ---------------------------------------------------------------- silu gate (+ resid)
 SILU_SHAPES = [(4096, 14336, 64), (256, 512, 64), (1000, 4096, 128), (77, 2048, 32),
-               (300, 28672, 64), (45, 36, 12)]
+               (300, 28672, 64), (45, 36, 12),
+               (500, 4096, 256), (64, 14336, 256)]   # group size the tensor-pipe kernel does not take
 
 
 @pytest.mark.parametrize("N,K,gs", SILU_SHAPES)
@@ -258,13 +260,24 @@ SMALLM_SHAPES = [(512, 1024, 64), (300, 4096, 32), (256, 14336, 128), (128, 2867
 
 
 @pytest.mark.parametrize("N,K,gs", SMALLM_SHAPES)
-@pytest.mark.parametrize("m", [1, 2, 3, 4, 5, 7, 8, 16, 32])
-def test_gemm_smallm(N, K, gs, m):
+@pytest.mark.parametrize("m", [1, 2, 3, 5, 8, 9, 16, 17, 32])
+def test_gemm_smallm_tensor_pipe(N, K, gs, m):
     W, g = make(8, N, K, gs)
     X = synth.activations(g, m, K)
     ref = oracle.gemm(*W.host, gs, X)
     assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_SMALLM), ref, f"smallm m={m} {N}x{K}")
     assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_AUTO), ref, f"auto m={m} {N}x{K}")
+
+
+@pytest.mark.parametrize("N,K,gs", SMALLM_SHAPES + [(300, 4096, 256)])
+@pytest.mark.parametrize("m", [1, 2, 4, 5, 16, 32])
+def test_gemm_smallm_fp32_pipes(N, K, gs, m):
+    W, g = make(9, N, K, gs)
+    X = synth.activations(g, m, K)
+    ref = oracle.gemm(*W.host, gs, X)
+    assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_SMALLM_FFMA), ref, f"smallm-ffma m={m} {N}x{K}")
+    if m > 8:
+        assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_AUTO), ref, f"auto m={m} {N}x{K}")
 
 
 @pytest.mark.parametrize("m", [1, 3, 9])

@@ -34,6 +34,7 @@ MLXQ_GEMM_AUTO = 0
 MLXQ_GEMM_ROWS = 1
 MLXQ_GEMM_SMALLM = 2
 MLXQ_GEMM_TCGEN05 = 3
+MLXQ_GEMM_SMALLM_FFMA = 4
 
 EXPORTS = ("mlxq_load", "mlxq_dequant", "mlxq_gemv", "mlxq_gemv_silu_gate",
            "mlxq_gemv_silu_gate_resid", "mlxq_gemm", "mlxq_gemm_with", "mlxq_release",

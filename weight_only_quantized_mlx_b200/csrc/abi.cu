@@ -522,14 +522,14 @@ int mlxq_gemv_silu_gate_resid(const mlxq_weight* w, const void* gate, const void
     return gemv_common(w, GEMV_SILU_RESID, nullptr, gate, up, x_resid, y, stream);
 }
 
-// m at or above this goes to the tensor-core kernel when it can take the shape.
-static const int64_t kTcMinM = 64;
-
+// Kernel choice by m: the weight-streaming kernels read every weight byte
+// once and are HBM-bound while the per-byte work fits the SM; beyond
+// kStreamMmaMaxM rows the tcgen05 kernel takes over.
 int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kernel, uint64_t stream) {
     WeightView v;
     int rc = check_weight(w, v);
     if (rc) return rc;
-    if (kernel < MLXQ_GEMM_AUTO || kernel > MLXQ_GEMM_TCGEN05)
+    if (kernel < MLXQ_GEMM_AUTO || kernel > MLXQ_GEMM_SMALLM_FFMA)
         return fail(MLXQ_ERR_INVALID_ARG, "unknown gemm kernel id %d", kernel);
     if (m == 0) return ok();
     const int64_t M = m;
@@ -539,10 +539,13 @@ int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32_t m, int
     if ((rc = check_out_vs_weight(y, M * v.N * 2, v))) return rc;
     if (v.N == 0) return ok();
     cudaStream_t s = as_stream(stream);
+    const bool x16 = (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
     int k = kernel;
     if (k == MLXQ_GEMM_AUTO) {
-        if (M >= kTcMinM && gemm_tc_supported(v, M, x, y)) k = MLXQ_GEMM_TCGEN05;
-        else if (M >= 2 && gemm_smallm_supported(v, M) && (reinterpret_cast<uintptr_t>(x) & 15u) == 0) k = MLXQ_GEMM_SMALLM;
+        if (M == 1) k = MLXQ_GEMM_ROWS;
+        else if (M <= kStreamMmaMaxM && stream_mma_supported(v, GEMV_PLAIN, M, x, nullptr, nullptr)) k = MLXQ_GEMM_SMALLM;
+        else if (gemm_tc_supported(v, M, x, y)) k = MLXQ_GEMM_TCGEN05;
+        else if (M <= kSmallMMax && x16 && gemm_smallm_supported(v, M)) k = MLXQ_GEMM_SMALLM_FFMA;
         else k = MLXQ_GEMM_ROWS;
     }
     switch (k) {
@@ -556,10 +559,16 @@ int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32_t m, int
             return ok();
         }
         case MLXQ_GEMM_SMALLM:
-            if (!gemm_smallm_supported(v, M) || (reinterpret_cast<uintptr_t>(x) & 15u) != 0)
-                return fail(MLXQ_ERR_UNSUPPORTED, "small-m kernel cannot take m=%lld, K=%lld, group_size=%lld",
+            if (M > kStreamMmaMaxM || !stream_mma_supported(v, GEMV_PLAIN, M, x, nullptr, nullptr))
+                return fail(MLXQ_ERR_UNSUPPORTED, "small-m tensor-pipe kernel cannot take m=%lld, K=%lld, group_size=%lld",
                             static_cast<long long>(M), static_cast<long long>(v.K), static_cast<long long>(v.gs));
-            return launch_status(launch_gemm_smallm(v, x, y, M, s), "small-m gemm launch");
+            return launch_status(launch_stream_mma(v, GEMV_PLAIN, M, x, nullptr, nullptr, nullptr, y, s),
+                                 "small-m gemm launch");
+        case MLXQ_GEMM_SMALLM_FFMA:
+            if (!gemm_smallm_supported(v, M) || !x16)
+                return fail(MLXQ_ERR_UNSUPPORTED, "small-m fp32 kernel cannot take m=%lld, K=%lld, group_size=%lld",
+                            static_cast<long long>(M), static_cast<long long>(v.K), static_cast<long long>(v.gs));
+            return launch_status(launch_gemm_smallm(v, x, y, M, s), "small-m fp32 gemm launch");
         default:
             if (!gemm_tc_supported(v, M, x, y))
                 return fail(MLXQ_ERR_UNSUPPORTED, "tensor-core kernel cannot take m=%lld, N=%lld, K=%lld, group_size=%lld",

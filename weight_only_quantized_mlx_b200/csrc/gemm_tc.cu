@@ -18,13 +18,9 @@
 // The accumulator is D[w_row][x_row] (TMEM lane = weight row), so each warp's
 // stores of one output row of Y are 32 consecutive BF16 values.  All pipeline
 // waits are bounded; no cluster multicast is used.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "device_common.cuh"
 #include "kernels.h"
+#include "tensor_map.h"
 
 namespace mlxq {
 namespace {
@@ -274,32 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---- host side -----------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-PFN_cuTensorMapEncodeTiled_v12000 encoder() {
-    std::call_once(g_encode_once, [] {
-        void* fn = nullptr;
-        cudaDriverEntryPointQueryResult q{};
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    });
-    return g_encode;
-}
-
-bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, void* base, uint64_t inner, uint64_t outer,
-               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
-    auto enc = encoder();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {box_inner, box_outer};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int pick_bn(int64_t m) {
     int64_t bn = (m + 31) / 32 * 32;
     return static_cast<int>(bn > 256 ? 256 : bn);
@@ -317,7 +287,7 @@ bool gemm_tc_supported(const WeightView& w, int64_t m, const void* X, const void
     int major = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device_info().device);
     if (major != 10) return false;
-    return encoder() != nullptr;
+    return tensor_maps_available();
 }
 
 cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream) {
@@ -349,11 +319,10 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
     p.tmem_cols = cols;
     p.status = device_status_ptr();
 
-    CUtensorMap tm_packed, tm_x;
-    if (!encode_2d(&tm_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<uint32_t*>(w.packed),
-                   static_cast<uint64_t>(w.K), static_cast<uint64_t>(w.N), static_cast<uint64_t>(w.K), kBK,
-                   kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
+    TensorMaps3 wm;
+    if (!weight_tensor_maps(w, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_NONE, 0, &wm)) return cudaErrorInvalidValue;
+    const CUtensorMap& tm_packed = wm.packed;
+    CUtensorMap tm_x;
     if (!encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(X), static_cast<uint64_t>(w.K),
                    static_cast<uint64_t>(m), static_cast<uint64_t>(w.K) * 2, kBK, static_cast<uint32_t>(p.BN),
                    CU_TENSOR_MAP_SWIZZLE_128B))

@@ -396,6 +396,8 @@ GemvParams base_params(const WeightView& w, const StreamPlan& pl) {
 cudaError_t launch_gemv(const WeightView& w, int mode, const void* x, const void* gate,
                         const void* up, const void* resid, void* y, cudaStream_t stream) {
     if (w.N == 0) return cudaSuccess;
+    if (stream_mma_supported(w, mode, 1, x, gate, up))
+        return launch_stream_mma(w, mode, 1, x, gate, up, resid, y, stream);
     const bool acts_aligned = (mode == GEMV_PLAIN) ? a16(x) : (a16(gate) && a16(up));
     const StreamPlan pl = plan_stream(w, acts_aligned, 1);
     GemvParams p = base_params(w, pl);

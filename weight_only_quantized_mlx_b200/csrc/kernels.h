@@ -55,6 +55,14 @@ cudaError_t launch_dequant(const WeightView& w, void* out, cudaStream_t stream);
 cudaError_t launch_gemv(const WeightView& w, int mode, const void* x, const void* gate,
                         const void* up, const void* resid, void* y, cudaStream_t stream);
 
+// Tensor-pipe stream kernel (mma.sync fragments) for m <= kStreamMmaMaxM:
+// gemv and its silu variants (m == 1) and small-m gemm (plain mode).
+constexpr int kStreamMmaMaxM = 32;
+bool stream_mma_supported(const WeightView& w, int mode, int64_t m, const void* x, const void* gate,
+                          const void* up);
+cudaError_t launch_stream_mma(const WeightView& w, int mode, int64_t m, const void* x, const void* gate,
+                              const void* up, const void* resid, void* y, cudaStream_t stream);
+
 // CUDA-core small-m gemm: Y [m, N] = X [m, K] W^T, 2 <= m <= kSmallMMax.
 constexpr int kSmallMMax = 32;
 bool gemm_smallm_supported(const WeightView& w, int64_t m);
