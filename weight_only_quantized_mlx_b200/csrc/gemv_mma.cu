@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t xs = sbase + static_cast<uint32_t>(S) * p.stage_bytes;  // activation staging
     auto stage_of = [&](int s) { return sbase + static_cast<uint32_t>(s) * p.stage_bytes; };
 
+    pdl_launch_dependents();  // the next kernel in the stream may be scheduled
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
@@ -123,6 +124,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&tm_packed);
             prefetch_tmap(&tm_scales);
             prefetch_tmap(&tm_biases);
+            // Warm L2 with the first stages while earlier kernels finish
+            // (L2 is coherent, so this is safe before the dependency wait;
+            // every load into shared memory comes after it).
+            for (int kb = 0; kb < S && kb < p.num_kb; ++kb) {
+                const int col0 = kb * kKB;
+                for (int b = 0; b < NB && col0 + 128 * b < p.K; ++b) tma_prefetch_l2_2d(&tm_packed, col0 + 128 * b, r0);
+                tma_prefetch_l2_2d(&tm_scales, kb * p.gpk, r0);
+                tma_prefetch_l2_2d(&tm_biases, kb * p.gpk, r0);
+            }
+            pdl_wait();
             const uint64_t pol = policy_evict_first();
             bool ok = true;
             for (int kb = 0; kb < p.num_kb; ++kb) {
@@ -146,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------- consumers ----------------
     const int ctid = threadIdx.x;  // 0 .. 32*kWarps-1
+    pdl_wait();  // activations, residual and the output belong to earlier work
     if (p.m == 1) {
         // stage the activation operand: x (plain) or the BF16 high/low split
         // of h = silu(gate)*up (silu variants: activation columns 0 and 1)
@@ -182,8 +194,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int box = warp % NB;
     const int sub = warp / NB;
-    // row pairs of this warp: sub, sub + kSub, ...
-    const int my_pairs = npair > sub ? (npair - sub + kSub - 1) / kSub : 0;
+    // Every warp runs the same trip counts (CTA-uniform), so the mma.sync loop
+    // has no divergent branches: a pair index past the CTA's rows re-reads the
+    // CTA's last pair, a box past K re-reads box 0 with zero activations, and
+    // those results are never stored.
+    const int pw_u = (npair + kSub - 1) / kSub;  // pairs per warp (uniform)
     float acc[PW][NT][4];
 #pragma unroll
     for (int j = 0; j < PW; ++j)
@@ -204,79 +219,89 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t sbo[PW];
 #pragma unroll
     for (int j = 0; j < PW; ++j) {
-        const int row = 16 * (sub + j * kSub) + g;
+        int pidx = sub + j * kSub;
+        if (pidx > npair - 1) pidx = npair - 1;
+        const int row = 16 * pidx + g;
         rowoff[j] = static_cast<uint32_t>(row) * 128u;
-        sbo[j] = static_cast<uint32_t>(row * p.gpk) * 2u;
+        sbo[j] = static_cast<uint32_t>(row * p.gpk + grp[0]) * 2u;
     }
+    const uint32_t sgrp1 = static_cast<uint32_t>(grp[1] - grp[0]) * 2u;
     const uint32_t sbo8 = static_cast<uint32_t>(8 * p.gpk) * 2u;
     // activation column this lane feeds (B column g of each 8-column tile)
     const bool plain1 = (p.m == 1 && MODE == GEMV_PLAIN);
-    const uint32_t xrow_off = (p.m == 1 && MODE != GEMV_PLAIN) ? 2u * static_cast<uint32_t>(g * p.K) : 0u;
+    // staged rows: x (plain, row 0) or h high/low (silu, rows 0 and 1); any
+    // other lane reads row 0 and discards it, so every load stays inside
+    const uint32_t xrow_off = (p.m == 1 && MODE != GEMV_PLAIN && g < 2) ? 2u * static_cast<uint32_t>(g * p.K) : 0u;
+    bool colv[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        const int col = 8 * t + g;
+        colv[t] = plain1 ? col == 0 : (p.m == 1 ? col < 2 : col < p.m);
+    }
     bool ok = true;
     for (int kb = 0; kb < p.num_kb; ++kb) {
         const int s = kb % S;
         if (ok) ok = mbar_wait(smem_u32(&full[s]), (kb / S) & 1, p.status);
         const int col0 = kb * kKB + box * 128;
-        if (col0 < p.K && my_pairs > 0) {
-            const uint32_t st = stage_of(s);
-            const uint32_t boxa = st + static_cast<uint32_t>(box) * p.box_bytes;
-            const uint32_t sca = st + NB * p.box_bytes;
-            const uint32_t bia = sca + p.sb_bytes;
+        const bool box_in = col0 < p.K;
+        const uint32_t st = stage_of(s);
+        const uint32_t boxa = st + static_cast<uint32_t>(box_in ? box : 0) * p.box_bytes;
+        const uint32_t sca = st + NB * p.box_bytes;
+        const uint32_t bia = sca + p.sb_bytes;
 #pragma unroll
-            for (int ci = 0; ci < 2; ++ci) {
-                const int kc = col0 + 16 * (tq + 4 * ci);
-                // B fragments: activation column (8 t + g) at this lane's 16 codes
-                uint32_t b[NT][8];
+        for (int ci = 0; ci < 2; ++ci) {
+            const int kc = col0 + 16 * (tq + 4 * ci);
+            const bool kin = box_in && kc < p.K;
+            const int kcs = kin ? kc : 0;  // a valid address when out of range
+            // B fragments: activation column (8 t + g) at this lane's 16 codes
+            uint32_t b[NT][8];
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    const int col = 8 * t + g;
-                    const bool live = kc < p.K && (plain1 ? col == 0 : (p.m == 1 ? col < 2 : col < p.m));
-                    if (live) {
-                        uint4 v0, v1;
-                        if (p.m == 1) {
-                            const uint32_t base = xs + xrow_off + 2u * static_cast<uint32_t>(kc);
-                            v0 = lds128(base);
-                            v1 = lds128(base + 16);
-                        } else {
-                            const uint16_t* xr = p.X + static_cast<int64_t>(col) * p.K + kc;
-                            v0 = ldg_nc_v4(xr);
-                            v1 = ldg_nc_v4(xr + 8);
-                        }
-                        b[t][0] = v0.x; b[t][1] = v0.y; b[t][2] = v0.z; b[t][3] = v0.w;
-                        b[t][4] = v1.x; b[t][5] = v1.y; b[t][6] = v1.z; b[t][7] = v1.w;
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) b[t][i] = 0u;
-                    }
+            for (int t = 0; t < NT; ++t) {
+                uint4 v0, v1;
+                if (p.m == 1) {
+                    const uint32_t base = xs + xrow_off + 2u * static_cast<uint32_t>(kcs);
+                    v0 = lds128(base);
+                    v1 = lds128(base + 16);
+                } else {
+                    const int colr = colv[t] ? 8 * t + g : 0;
+                    const uint16_t* xr = p.X + static_cast<int64_t>(colr) * p.K + kcs;
+                    v0 = ldg_nc_v4(xr);
+                    v1 = ldg_nc_v4(xr + 8);
                 }
-                // row pairs in groups of two: load both, then interleave the MMAs
+                const bool live = kin && colv[t];
+                b[t][0] = live ? v0.x : 0u; b[t][1] = live ? v0.y : 0u;
+                b[t][2] = live ? v0.z : 0u; b[t][3] = live ? v0.w : 0u;
+                b[t][4] = live ? v1.x : 0u; b[t][5] = live ? v1.y : 0u;
+                b[t][6] = live ? v1.z : 0u; b[t][7] = live ? v1.w : 0u;
+            }
+            const uint32_t sgo = ci ? sgrp1 : 0u;
+            // row pairs in groups of two: load both, then interleave the MMAs
 #pragma unroll
-                for (int j0 = 0; j0 < PW; j0 += 2) {
+            for (int j0 = 0; j0 < PW; j0 += 2) {
+                if (j0 < pw_u) {  // CTA-uniform
                     uint4 wlo[2], whi[2];
                     float2 slo[2], blo[2], shi[2], bhi[2];
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj) {
-                        const int j = j0 + jj;
-                        if (j < PW && j < my_pairs) {
-                            wlo[jj] = lds128(boxa + rowoff[j] + swz[ci]);
-                            whi[jj] = lds128(boxa + rowoff[j] + 8u * 128u + swz[ci]);
-                            const uint32_t sidx = sbo[j] + static_cast<uint32_t>(grp[ci]) * 2u;
-                            const float s0 = bf16_bits_to_f32(lds16(sca + sidx));
-                            const float b0 = bf16_bits_to_f32(lds16(bia + sidx));
-                            const float s1 = bf16_bits_to_f32(lds16(sca + sidx + sbo8));
-                            const float b1 = bf16_bits_to_f32(lds16(bia + sidx + sbo8));
-                            slo[jj] = make_float2(s0, s0);
-                            blo[jj] = make_float2(b0, b0);
-                            shi[jj] = make_float2(s1, s1);
-                            bhi[jj] = make_float2(b1, b1);
-                        }
+                        const int j = (j0 + jj < PW) ? j0 + jj : j0;
+                        wlo[jj] = lds128(boxa + rowoff[j] + swz[ci]);
+                        whi[jj] = lds128(boxa + rowoff[j] + 8u * 128u + swz[ci]);
+                        const uint32_t sidx = sbo[j] + sgo;
+                        const float s0 = bf16_bits_to_f32(lds16(sca + sidx));
+                        const float b0 = bf16_bits_to_f32(lds16(bia + sidx));
+                        const float s1 = bf16_bits_to_f32(lds16(sca + sidx + sbo8));
+                        const float b1 = bf16_bits_to_f32(lds16(bia + sidx + sbo8));
+                        slo[jj] = make_float2(s0, s0);
+                        blo[jj] = make_float2(b0, b0);
+                        shi[jj] = make_float2(s1, s1);
+                        bhi[jj] = make_float2(b1, b1);
                     }
 #pragma unroll
                     for (int w4 = 0; w4 < 4; ++w4) {
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
                             const int j = j0 + jj;
-                            if (j < PW && j < my_pairs) {
+                            if (j < PW && (jj == 0 || j0 + 1 < pw_u)) {  // CTA-uniform
                                 const uint32_t ul = w4 == 0 ? wlo[jj].x : w4 == 1 ? wlo[jj].y : w4 == 2 ? wlo[jj].z : wlo[jj].w;
                                 const uint32_t uh = w4 == 0 ? whi[jj].x : w4 == 1 ? whi[jj].y : w4 == 2 ? whi[jj].z : whi[jj].w;
                                 uint32_t a0, a2, a1, a3;
@@ -294,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
     }
+    const int my_pairs = npair > sub ? (npair - sub + kSub - 1) / kSub : 0;
 
     // ---- cross-warp sum (fixed order) in the freed stage area ----
     named_bar_sync(1, kWarps * 32);  // every warp is done with the stage buffers
@@ -351,7 +377,8 @@ cudaError_t launch_t(const TensorMaps3& tm, const MmaParams& p, int grid, size_t
     static std::atomic<int> configured[64];
     cudaError_t e = ensure_dynamic_smem(kern, smem, configured);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, stream>>>(tm.packed, tm.scales, tm.biases, p);
+    e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, tm.packed, tm.scales, tm.biases, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

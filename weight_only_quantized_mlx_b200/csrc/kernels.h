@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 namespace mlxq {
 
@@ -46,6 +47,25 @@ cudaError_t ensure_dynamic_smem(Kernel kern, size_t bytes, std::atomic<int> (&co
         }
     }
     return e;
+}
+
+// Launch with programmatic stream serialization (PDL): the kernel may start
+// while the previous one in the stream finishes; kernels launched this way
+// call griddepcontrol.wait before touching any input or output in memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // mlx_int8_dequant: out [N, K] bf16.
