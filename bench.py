@@ -70,7 +70,10 @@ def profile_traffic(kernel_tag: str, source_files):
     for line in open(path):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
+            v = v.strip()
+            if v.startswith("`") and v.count("`") >= 2:
+                v = v[1:v.index("`", 1)]  # the first backticked token
+            vals[k.strip()] = v
     if vals.get("source_sha256") != h.hexdigest()[:16]:
         return None
     try:
@@ -257,7 +260,7 @@ def run_gpu(args):
     e2e_value = total_bytes / (ms_e2e * 1e-3) / 1e9
     achieved = per_launch / (ms * 1e-3 / N_PAIRS) / 1e9
     traffic = profile_traffic("gemv_decode_4096x4096_gs64", [
-        "weight_only_quantized_mlx_b200/csrc/gemv.cu",
+        "weight_only_quantized_mlx_b200/csrc/gemv_mma.cu",
         "weight_only_quantized_mlx_b200/csrc/device_common.cuh"])
     out = {
         "metric": "W8 group-affine GEMV HBM GB/s (% of peak) at m=1; gemm TFLOP/s at m=4096",
@@ -285,7 +288,7 @@ def run_gpu(args):
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-            "peak_source": peaks["source"], "kernel": "k_gemv_stream (mlx_int8_gemv)",
+            "peak_source": peaks["source"], "kernel": "k_stream_mma (mlx_int8_gemv)",
         },
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": 2 * D_K * N_PAIRS, "d2h_bytes_per_step": 2 * D_N * N_PAIRS},

@@ -104,8 +104,9 @@ MLXQ_API int mlxq_gemv(const mlxq_weight* w, const void* x, void* y, uint64_t st
 /*
  * mlxq_gemv_silu_gate (page: MlxInt8Weight::gemv_silu_gate, kernel
  * mlx_int8_gemv_silu_gate).  y = W (silu(gate) * up), silu(t) = t/(1+e^-t),
- * in one launch; silu(gate)*up is formed in registers and never written to
- * memory.  gate, up: BF16 [K]; y: BF16 [N].
+ * in one launch; the product silu(gate)*up exists only on chip (registers and
+ * shared memory), it is not stored to global memory.  gate, up: BF16 [K];
+ * y: BF16 [N].
  */
 MLXQ_API int mlxq_gemv_silu_gate(const mlxq_weight* w, const void* gate, const void* up, void* y,
                         uint64_t stream);

@@ -12,7 +12,7 @@
 //    transaction count; consumers free a stage with an mbarrier arrive.
 //  * Consumer thread t owns the same 16-code chunks of every row (chunk
 //    c = t + j*T), so its slice of h = x (or silu(gate)*up, fp32, computed
-//    once in registers and never written to memory) is loaded once.
+//    once in registers, not stored to global memory) is loaded once.
 //  * Per chunk: unpack 16 codes (byte -> fp32 through the 2^23 exponent
 //    trick), w = fma(s, q, b) in fp32, round to BF16 (so W equals the BF16
 //    weight the page's dequantize_to produces), fp32 FMA with h, using the
