@@ -25,19 +25,30 @@
 namespace mlxq {
 namespace {
 
-constexpr int kBM = 128;                // weight rows per tile (MMA M)
+constexpr int kBM = 256;                // weight rows per tile: two MMA M=128 halves
+constexpr int kHM = 128;                // rows per MMA half
 constexpr int kBK = 64;                 // k per stage: one 128-byte row of BF16
 constexpr int kDequantWarps = 8;
-constexpr int kThreads = (2 + kDequantWarps) * 32;
-constexpr uint32_t kStageA = kBM * 128;  // BF16 A tile
-constexpr uint32_t kStageP = kBM * kBK;  // packed codes
+constexpr int kEpilogueWarps = 8;       // two per TMEM lane quadrant (one per accumulator half)
+constexpr int kFirstDequant = 3;        // warps: 0 X producer, 1 MMA, 2 weight producer
+constexpr int kFirstEpilogue = kFirstDequant + kDequantWarps;
+constexpr int kThreads = (kFirstEpilogue + kEpilogueWarps) * 32;
+constexpr uint32_t kStageA = kBM * 128;  // BF16 A tile (two 128-row halves)
+constexpr uint32_t kStageP = kBM * kBK;  // packed codes of one k-block
+constexpr int kSbGroups = 8;             // scale groups per scale/bias box (16 bytes per row)
+constexpr uint32_t kStageSB = kBM * kSbGroups * 2;  // one box of scales (or biases)
+constexpr int kXBoxRows = 32;            // activation rows per TMA box
+constexpr int kSP = 3;                   // packed-code slots
+constexpr int kSSB = 2;                  // scale/bias slots
 
 struct TcParams {
-    const uint16_t* scales;
-    const uint16_t* biases;
     uint16_t* Y;
     int N, K, G, gs, m;
     int BN, S, num_kb;
+    int sg;          // k-blocks covered by one scale/bias box (8 * gs / 64)
+    int sb_tma;      // 1: scales/biases by TMA boxes; 0 (rows not 16-byte multiples): direct loads
+    const uint16_t* scales;
+    const uint16_t* biases;
     uint32_t stage_bytes, idesc, tmem_cols;
     unsigned int* status;
 };
@@ -102,170 +113,276 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
     return d;
 }
 
+// Persistent: CTA b processes tiles b, b + gridDim.x, ... (weight-row tile
+// fastest).  A tile is 256 weight rows x BN activation rows: two M=128 MMAs per
+// 16-wide k step share the activation (B) tile.  All operand bytes arrive by
+// TMA: the activation tile into the (A, X) stage ring, the packed codes into
+// their own ring, and the scales/biases as 8-group boxes into a third ring;
+// the dequant warps read only shared memory.  The two fp32 accumulators fill
+// TMEM (2 x BN <= 512 columns).
 __global__ void __launch_bounds__(kThreads, 1)
-    k_gemm_tc(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_x,
+    k_gemm_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_packed,
+              const __grid_constant__ CUtensorMap tm_scales, const __grid_constant__ CUtensorMap tm_biases,
               const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-byte aligned (swizzle atoms)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.S;
-    const int n0 = blockIdx.x * kBM;
-    const int m0 = blockIdx.y * p.BN;
     const uint32_t stage_x = static_cast<uint32_t>(p.BN) * 128u;
+    const int tiles_n = (p.N + kBM - 1) / kBM;
+    const int tiles_m = (p.m + p.BN - 1) / p.BN;
+    const int num_tiles = tiles_n * tiles_m;
+    const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int sb_per_tile = (p.num_kb + p.sg - 1) / p.sg;
 
-    uint64_t* pfull = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * p.stage_bytes);
-    uint64_t* full = pfull + S;
-    uint64_t* empty = full + S;
-    uint64_t* accum = empty + S;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+    // shared memory: S (A, X) stages | kSP packed slots | kSSB (scales, biases) slots | barriers
     const uint32_t sbase = smem_u32(smem);
+    const uint32_t p_base = sbase + static_cast<uint32_t>(S) * p.stage_bytes;
+    const uint32_t sb_base = p_base + kSP * kStageP;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * p.stage_bytes + kSP * kStageP +
+                                                 kSSB * 2 * kStageSB);
+    uint64_t* empty = full + S;
+    uint64_t* pfull = empty + S;
+    uint64_t* pempty = pfull + kSP;
+    uint64_t* sbfull = pempty + kSP;
+    uint64_t* sbempty = sbfull + kSSB;
+    uint64_t* acc_full = sbempty + kSSB;
+    uint64_t* acc_empty = acc_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
     auto A_of = [&](int s) { return sbase + static_cast<uint32_t>(s) * p.stage_bytes; };
     auto X_of = [&](int s) { return A_of(s) + kStageA; };
-    auto P_of = [&](int s) { return X_of(s) + stage_x; };
+    auto P_of = [&](int s) { return p_base + static_cast<uint32_t>(s) * kStageP; };
+    auto SC_of = [&](int s) { return sb_base + static_cast<uint32_t>(s) * 2u * kStageSB; };
+    auto BI_of = [&](int s) { return SC_of(s) + kStageSB; };
+    auto tile_nm = [&](int t, int& n0, int& m0) {
+        const int tile = blockIdx.x + t * gridDim.x;
+        n0 = (tile % tiles_n) * kBM;
+        m0 = (tile / tiles_n) * p.BN;
+    };
 
+    pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&pfull[s]), 1);
             mbar_init(smem_u32(&full[s]), 1 + kDequantWarps);
             mbar_init(smem_u32(&empty[s]), 1);
         }
-        mbar_init(smem_u32(accum), 1);
+        for (int s = 0; s < kSP; ++s) {
+            mbar_init(smem_u32(&pfull[s]), 1);
+            mbar_init(smem_u32(&pempty[s]), kDequantWarps);
+        }
+        for (int s = 0; s < kSSB; ++s) {
+            mbar_init(smem_u32(&sbfull[s]), 1);
+            mbar_init(smem_u32(&sbempty[s]), kDequantWarps);
+        }
+        mbar_init(smem_u32(acc_full), 1);
+        mbar_init(smem_u32(acc_empty), kEpilogueWarps);
         mbar_fence_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+        tmem_alloc(smem_u32(tmem_slot), 2 * p.tmem_cols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_d = *tmem_slot;
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // activations, weights and Y belong to earlier work
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- activation producer ----------------
+        if (lane == 0) {
+            prefetch_tmap(&tm_x);
+            const uint64_t pol = policy_evict_last();  // each activation tile serves every weight tile
+            bool ok = true;
+            int it = 0;
+            for (int t = 0; t < my_tiles; ++t) {
+                int n0, m0;
+                tile_nm(t, n0, m0);
+                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                    const int s = it % S;
+                    if (it >= S && ok) ok = mbar_wait(smem_u32(&empty[s]), ((it / S) - 1) & 1, p.status);
+                    mbar_arrive_expect_tx(smem_u32(&full[s]), stage_x);
+                    for (int r = 0; r < p.BN; r += kXBoxRows)
+                        tma_load_2d(X_of(s) + static_cast<uint32_t>(r) * 128u, &tm_x, kb * kBK, m0 + r,
+                                    smem_u32(&full[s]), pol);
+                }
+            }
+        }
+    } else if (warp == 2) {
+        // ---------------- weight producer: packed codes, scales, biases ----------------
         if (lane == 0) {
             prefetch_tmap(&tm_packed);
-            prefetch_tmap(&tm_x);
-            const uint64_t pol_w = policy_evict_first();
-            const uint64_t pol_x = policy_evict_last();
+            prefetch_tmap(&tm_scales);
+            prefetch_tmap(&tm_biases);
+            const uint64_t pol = policy_evict_last();  // each weight tile serves every activation tile
             bool ok = true;
-            for (int kb = 0; kb < p.num_kb; ++kb) {
-                const int s = kb % S;
-                if (kb >= S && ok) ok = mbar_wait(smem_u32(&empty[s]), ((kb / S) - 1) & 1, p.status);
-                mbar_arrive_expect_tx(smem_u32(&pfull[s]), kStageP);
-                tma_load_2d(P_of(s), &tm_packed, kb * kBK, n0, smem_u32(&pfull[s]), pol_w);
-                mbar_arrive_expect_tx(smem_u32(&full[s]), stage_x);
-                tma_load_2d(X_of(s), &tm_x, kb * kBK, m0, smem_u32(&full[s]), pol_x);
+            int it = 0, sbi = 0;
+            for (int t = 0; t < my_tiles; ++t) {
+                int n0, m0;
+                tile_nm(t, n0, m0);
+                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                    if (p.sb_tma && kb % p.sg == 0) {  // a new scale/bias box for the next sg k-blocks
+                        const int ss = sbi % kSSB;
+                        if (sbi >= kSSB && ok) ok = mbar_wait(smem_u32(&sbempty[ss]), ((sbi / kSSB) - 1) & 1, p.status);
+                        mbar_arrive_expect_tx(smem_u32(&sbfull[ss]), 2u * kStageSB);
+                        const int g0 = (kb / p.sg) * kSbGroups;
+                        tma_load_2d(SC_of(ss), &tm_scales, g0, n0, smem_u32(&sbfull[ss]), pol);
+                        tma_load_2d(BI_of(ss), &tm_biases, g0, n0, smem_u32(&sbfull[ss]), pol);
+                        ++sbi;
+                    }
+                    const int sp = it % kSP;
+                    if (it >= kSP && ok) ok = mbar_wait(smem_u32(&pempty[sp]), ((it / kSP) - 1) & 1, p.status);
+                    mbar_arrive_expect_tx(smem_u32(&pfull[sp]), kStageP);
+                    tma_load_2d(P_of(sp), &tm_packed, kb * kBK, n0, smem_u32(&pfull[sp]), pol);
+                }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             bool ok = true;
-            for (int kb = 0; kb < p.num_kb; ++kb) {
-                const int s = kb % S;
-                if (ok) ok = mbar_wait(smem_u32(&full[s]), (kb / S) & 1, p.status);
+            int it = 0;
+            for (int t = 0; t < my_tiles; ++t) {
+                // the epilogue must have drained the accumulators (previous tile)
+                if (t >= 1 && ok) ok = mbar_wait(smem_u32(acc_empty), (t - 1) & 1, p.status);
                 tc_fence_after();
-                const uint64_t ad = sw128_kmajor_desc(A_of(s));
-                const uint64_t bd = sw128_kmajor_desc(X_of(s));
+                const uint32_t d0 = tmem_base, d1 = tmem_base + p.tmem_cols;
+                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                    const int s = it % S;
+                    if (ok) ok = mbar_wait(smem_u32(&full[s]), (it / S) & 1, p.status);
+                    tc_fence_after();
+                    const uint64_t a0 = sw128_kmajor_desc(A_of(s));
+                    const uint64_t a1 = sw128_kmajor_desc(A_of(s) + kHM * 128u);
+                    const uint64_t bd = sw128_kmajor_desc(X_of(s));
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk) {
-                    // advance 16 BF16 (32 bytes) along K inside the swizzled row
-                    umma_bf16(tmem_d, ad + 2u * kk, bd + 2u * kk, p.idesc, (kb | kk) != 0);
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        // advance 16 BF16 (32 bytes) along K inside the swizzled rows
+                        const uint32_t acc = (kb | kk) != 0;
+                        umma_bf16(d0, a0 + 2u * kk, bd + 2u * kk, p.idesc, acc);
+                        umma_bf16(d1, a1 + 2u * kk, bd + 2u * kk, p.idesc, acc);
+                    }
+                    umma_commit(smem_u32(&empty[s]));
                 }
-                umma_commit(smem_u32(&empty[s]));
+                umma_commit(smem_u32(acc_full));
             }
-            umma_commit(smem_u32(accum));
         }
         __syncwarp();
-    } else {
-        // ---------------- dequant, then epilogue ----------------
-        const int dt = (warp - 2) * 32 + lane;  // 0 .. 255
-        const int chunk = dt & 3;               // 16-code chunk of the 64-code k-block
-        const int rbase = dt >> 2;              // rows rbase and rbase + 64
+    } else if (warp < kFirstEpilogue) {
+        // ---------------- dequant: packed codes -> BF16 A operand ----------------
+        const int dt = (warp - kFirstDequant) * 32 + lane;  // 0 .. 255
+        const int chunk = dt & 3;                           // 16-code chunk of the 64-code k-block
+        const int rbase = dt >> 2;                          // rows rbase + 64 i, i = 0..3
         bool ok = true;
-        // scale/bias of the next k-block, loaded one block ahead
-        float sc[2], bi[2];
-        auto load_sb = [&](int kb, float (&s_)[2], float (&b_)[2]) {
-            int g = (kb * kBK + chunk * 16) / p.gs;
-            if (g > p.G - 1) g = p.G - 1;
+        const float2 m2 = make_float2(-kMagic, -kMagic);
+        int it = 0, sbi = 0;
+        for (int t = 0; t < my_tiles; ++t) {
+            for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                const int ss = sbi % kSSB;
+                if (p.sb_tma && kb % p.sg == 0 && ok) ok = mbar_wait(smem_u32(&sbfull[ss]), (sbi / kSSB) & 1, p.status);
+                const int sp = it % kSP;
+                if (ok) ok = mbar_wait(smem_u32(&pfull[sp]), (it / kSP) & 1, p.status);
+                // this thread's codes and the scale/bias of their group, for 4 rows
+                const int gl = ((kb % p.sg) * kBK + chunk * 16) / p.gs;  // group within the box
+                uint4 wq[4];
+                float2 s2[4], b2[4];
+                int n0 = 0, m0 = 0;
+                if (!p.sb_tma) tile_nm(t, n0, m0);
+                const int k0 = kb * kBK + chunk * 16;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int n = n0 + rbase + 64 * i;
-                if (n < p.N) {
-                    s_[i] = bf16_bits_to_f32(__ldg(p.scales + static_cast<int64_t>(n) * p.G + g));
-                    b_[i] = bf16_bits_to_f32(__ldg(p.biases + static_cast<int64_t>(n) * p.G + g));
-                } else {
-                    s_[i] = 0.f;
-                    b_[i] = 0.f;
+                for (int i = 0; i < 4; ++i) {
+                    const int row = rbase + 64 * i;
+                    wq[i] = lds128(P_of(sp) + static_cast<uint32_t>(row * kBK + chunk * 16));
+                    float sv = 0.f, bv = 0.f;
+                    if (p.sb_tma) {
+                        const uint32_t so = static_cast<uint32_t>(row * kSbGroups + gl) * 2u;
+                        sv = bf16_bits_to_f32(lds16(SC_of(ss) + so));
+                        bv = bf16_bits_to_f32(lds16(BI_of(ss) + so));
+                    } else if (n0 + row < p.N && k0 < p.K) {
+                        const int64_t gi = static_cast<int64_t>(n0 + row) * p.G + k0 / p.gs;
+                        sv = bf16_bits_to_f32(__ldg(p.scales + gi));
+                        bv = bf16_bits_to_f32(__ldg(p.biases + gi));
+                    }
+                    s2[i] = make_float2(sv, sv);
+                    b2[i] = make_float2(bv, bv);
                 }
-            }
-        };
-        load_sb(0, sc, bi);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-            const int s = kb % S;
-            float scn[2] = {0.f, 0.f}, bin[2] = {0.f, 0.f};
-            if (kb + 1 < p.num_kb) load_sb(kb + 1, scn, bin);
-            if (ok) ok = mbar_wait(smem_u32(&pfull[s]), (kb / S) & 1, p.status);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int row = rbase + 64 * i;
-                const uint4 wq = lds128(P_of(s) + row * kBK + chunk * 16);
-                const uint32_t words[4] = {wq.x, wq.y, wq.z, wq.w};
-                uint32_t o[8];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t u = words[j];
-                    const float q0 = code_magic<0>(u) - kMagic, q1 = code_magic<1>(u) - kMagic;
-                    const float q2 = code_magic<2>(u) - kMagic, q3 = code_magic<3>(u) - kMagic;
-                    o[2 * j] = pack_bf16x2(__fmaf_rn(sc[i], q0, bi[i]), __fmaf_rn(sc[i], q1, bi[i]));
-                    o[2 * j + 1] = pack_bf16x2(__fmaf_rn(sc[i], q2, bi[i]), __fmaf_rn(sc[i], q3, bi[i]));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&pempty[sp]));  // packed slot read
+                if (p.sb_tma && (kb % p.sg == p.sg - 1 || kb == p.num_kb - 1)) {
+                    if (lane == 0) mbar_arrive(smem_u32(&sbempty[ss]));  // last use of this box
+                    ++sbi;
                 }
-                // logical 16-byte chunks 2*chunk and 2*chunk+1 of this 128-byte row,
-                // placed by the 128-byte swizzle (chunk index ^ row % 8)
-                const uint32_t rowa = A_of(s) + static_cast<uint32_t>(row) * 128u;
-                const uint32_t sw = static_cast<uint32_t>(row & 7);
-                sts128(rowa + (((2u * chunk) ^ sw) << 4), o[0], o[1], o[2], o[3]);
-                sts128(rowa + (((2u * chunk + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+                const int s = it % S;
+                // the MMA that last read this stage's A tile must be done
+                if (it >= S && ok) ok = mbar_wait(smem_u32(&empty[s]), ((it / S) - 1) & 1, p.status);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int row = rbase + 64 * i;  // 0..255: half row >> 7
+                    const uint32_t words[4] = {wq[i].x, wq[i].y, wq[i].z, wq[i].w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t u = words[j];
+                        const float2 q01 = __fadd2_rn(make_float2(code_magic<0>(u), code_magic<1>(u)), m2);
+                        const float2 q23 = __fadd2_rn(make_float2(code_magic<2>(u), code_magic<3>(u)), m2);
+                        const float2 w01 = __ffma2_rn(q01, s2[i], b2[i]);
+                        const float2 w23 = __ffma2_rn(q23, s2[i], b2[i]);
+                        o[2 * j] = pack_bf16x2(w01.x, w01.y);
+                        o[2 * j + 1] = pack_bf16x2(w23.x, w23.y);
+                    }
+                    // logical 16-byte chunks 2*chunk and 2*chunk+1 of this 128-byte row,
+                    // placed by the 128-byte swizzle (chunk index ^ row % 8)
+                    const uint32_t rowa = A_of(s) + static_cast<uint32_t>(row) * 128u;
+                    const uint32_t sw = static_cast<uint32_t>(row & 7);
+                    sts128(rowa + (((2u * chunk) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+                    sts128(rowa + (((2u * chunk + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&full[s]));
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&full[s]));
-            sc[0] = scn[0];
-            sc[1] = scn[1];
-            bi[0] = bin[0];
-            bi[1] = bin[1];
         }
-        // epilogue: TMEM lane = weight row, column = activation row
-        if (ok) ok = mbar_wait(smem_u32(accum), 0, p.status);
-        tc_fence_after();
-        const int q = warp & 3;                // TMEM lane quadrant this warp may access
-        const int half = (warp - 2) >> 2;      // which half of the BN columns
-        const int row = q * 32 + lane;
-        const int n = n0 + row;
-        const int cols = p.BN >> 1;
-        for (int c0 = half * cols; c0 < (half + 1) * cols; c0 += 16) {
-            uint32_t r[16];
-            tmem_ld16(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c0), r);
-            tmem_ld_wait();
-            if (n < p.N) {
+    } else {
+        // ---------------- epilogue: TMEM -> BF16 Y ----------------
+        // TMEM lane = weight row within a half, column = activation row
+        const int ew = warp - kFirstEpilogue;  // 0..7
+        const int q = warp & 3;                // lane quadrant this warp may access
+        const int half = ew >> 2;              // accumulator half
+        const int row = half * kHM + q * 32 + lane;
+        bool ok = true;
+        for (int t = 0; t < my_tiles; ++t) {
+            int n0, m0;
+            tile_nm(t, n0, m0);
+            if (ok) ok = mbar_wait(smem_u32(acc_full), t & 1, p.status);
+            tc_fence_after();
+            const uint32_t d = tmem_base + static_cast<uint32_t>(half) * p.tmem_cols +
+                               (static_cast<uint32_t>(q * 32) << 16);
+            const int n = n0 + row;
+            const int cols = p.m - m0 < p.BN ? p.m - m0 : p.BN;
+            for (int c0 = 0; c0 < cols; c0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(d + static_cast<uint32_t>(c0), r);
+                tmem_ld_wait();
+                if (n < p.N) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int i = m0 + c0 + j;
-                    if (i < p.m) {
-                        const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
-                        p.Y[static_cast<int64_t>(i) * p.N + n] = *reinterpret_cast<const uint16_t*>(&v);
+                    for (int j = 0; j < 16; ++j) {
+                        if (c0 + j < cols) {
+                            const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
+                            p.Y[static_cast<int64_t>(m0 + c0 + j) * p.N + n] = *reinterpret_cast<const uint16_t*>(&v);
+                        }
                     }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(acc_empty));
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_d, p.tmem_cols);
+        tmem_dealloc(tmem_base, 2 * p.tmem_cols);
     }
 }
 
@@ -293,8 +410,6 @@ bool gemm_tc_supported(const WeightView& w, int64_t m, const void* X, const void
 cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream) {
     const DeviceInfo& dev = device_info();
     TcParams p{};
-    p.scales = w.scales;
-    p.biases = w.biases;
     p.Y = static_cast<uint16_t*>(Y);
     p.N = static_cast<int>(w.N);
     p.K = static_cast<int>(w.K);
@@ -303,9 +418,13 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
     p.m = static_cast<int>(m);
     p.BN = pick_bn(m);
     p.num_kb = static_cast<int>((w.K + kBK - 1) / kBK);
-    p.stage_bytes = kStageA + static_cast<uint32_t>(p.BN) * 128u + kStageP;
-    const size_t tail = 1024 /*alignment slack*/ + 64 * sizeof(uint64_t);
-    int S = static_cast<int>((static_cast<size_t>(dev.max_smem_optin) - tail) / p.stage_bytes);
+    p.sg = static_cast<int>(kSbGroups * w.gs / kBK);
+    p.sb_tma = (w.G % 8 == 0) ? 1 : 0;
+    p.scales = w.scales;
+    p.biases = w.biases;
+    p.stage_bytes = kStageA + static_cast<uint32_t>(p.BN) * 128u;
+    const size_t fixed = 1024 /*alignment slack*/ + kSP * kStageP + kSSB * 2 * kStageSB + 64 * sizeof(uint64_t);
+    int S = static_cast<int>((static_cast<size_t>(dev.max_smem_optin) - fixed) / p.stage_bytes);
     if (S > 6) S = 6;
     if (S < 2) return cudaErrorInvalidValue;
     p.S = S;
@@ -313,28 +432,30 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
               | (1u << 7)                                 // A: BF16
               | (1u << 10)                                // B: BF16
               | (static_cast<uint32_t>(p.BN >> 3) << 17)  // N
-              | (static_cast<uint32_t>(kBM >> 4) << 24);  // M
+              | (static_cast<uint32_t>(kHM >> 4) << 24);  // M
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(p.BN)) cols <<= 1;
-    p.tmem_cols = cols;
+    p.tmem_cols = cols;  // per accumulator half; two halves allocated
     p.status = device_status_ptr();
 
     TensorMaps3 wm;
-    if (!weight_tensor_maps(w, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_NONE, 0, &wm)) return cudaErrorInvalidValue;
-    const CUtensorMap& tm_packed = wm.packed;
+    if (!weight_tensor_maps(w, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_NONE, p.sb_tma ? kSbGroups : 0, &wm))
+        return cudaErrorInvalidValue;
     CUtensorMap tm_x;
     if (!encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(X), static_cast<uint64_t>(w.K),
-                   static_cast<uint64_t>(m), static_cast<uint64_t>(w.K) * 2, kBK, static_cast<uint32_t>(p.BN),
+                   static_cast<uint64_t>(m), static_cast<uint64_t>(w.K) * 2, kBK, kXBoxRows,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
 
-    const size_t smem = static_cast<size_t>(S) * p.stage_bytes + tail;
+    const size_t smem = static_cast<size_t>(S) * p.stage_bytes + fixed;
     static std::atomic<int> configured[64];
     cudaError_t e = ensure_dynamic_smem(k_gemm_tc, smem, configured);
     if (e != cudaSuccess) return e;
-    const dim3 grid(static_cast<unsigned>((w.N + kBM - 1) / kBM), static_cast<unsigned>((m + p.BN - 1) / p.BN));
-    if (grid.y > 65535) return cudaErrorInvalidValue;
-    k_gemm_tc<<<grid, kThreads, smem, stream>>>(tm_packed, tm_x, p);
+    const int64_t tiles = ((w.N + kBM - 1) / kBM) * ((m + p.BN - 1) / p.BN);
+    if (tiles > (1ll << 31) - 1) return cudaErrorInvalidValue;
+    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    e = launch_pdl(k_gemm_tc, dim3(grid), dim3(kThreads), smem, stream, tm_x, wm.packed, wm.scales, wm.biases, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
