@@ -372,22 +372,30 @@ def measure_rows(mq, torch, synth, dev, stream, dec_weights, peaks, args):
                                             "us": round(ms * 1e3, 2)}
         w.release()
 
-    # prefill gemm at m = 4096 (tensor cores when the kernel takes the shape)
+    # prefill gemm (tensor cores): m = 4096 fills every SM with whole tiles;
+    # m = 512 and 128 have fewer tiles than SMs, so each tile's K is split
+    # (three weight copies, 183 MB, taken in turn: larger than L2)
     for (N, K) in ((4096, 14336), (14336, 4096)):
-        w = upload_weight(mq, *synth.weight(synth.rng(4000 + N), N, K, 64), 64)
-        m = 4096
-        X = torch.randn(m, K, device=dev).to(torch.bfloat16)
-        Y = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
-        try:
-            ms = time_region(lambda: mq.mlxq_gemm_with(w.handle, X, Y, m, mq.MLXQ_GEMM_TCGEN05, stream),
-                             steps, warm, stream, 1)
-            tf = 2 * m * N * K / (ms * 1e-3) / 1e12
-            rows[f"prefill_{N}x{K}_m{m}"] = {"value": round(tf, 1), "unit": "TFLOP/s",
-                                             "frac_bf16": round(tf / peaks["bf16_tflops"], 4),
-                                             "ms": round(ms, 4)}
-        except mq.MlxqError as e:
-            rows[f"prefill_{N}x{K}_m{m}"] = {"value": None, "unit": "TFLOP/s", "unavailable": str(e)}
-        w.release()
+        ws = [upload_weight(mq, *synth.weight(synth.rng(4000 + N + i), N, K, 64), 64) for i in range(3)]
+        for m in (4096, 512, 128):
+            X = torch.randn(m, K, device=dev).to(torch.bfloat16)
+            Y = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
+            turn = [0]
+
+            def call():
+                w = ws[turn[0] % len(ws)]
+                turn[0] += 1
+                mq.mlxq_gemm_with(w.handle, X, Y, m, mq.MLXQ_GEMM_TCGEN05, stream)
+            try:
+                ms = time_region(call, steps, warm, stream, 1)
+                tf = 2 * m * N * K / (ms * 1e-3) / 1e12
+                rows[f"prefill_{N}x{K}_m{m}"] = {"value": round(tf, 1), "unit": "TFLOP/s",
+                                                 "frac_bf16": round(tf / peaks["bf16_tflops"], 4),
+                                                 "ms": round(ms, 4)}
+            except mq.MlxqError as e:
+                rows[f"prefill_{N}x{K}_m{m}"] = {"value": None, "unit": "TFLOP/s", "unavailable": str(e)}
+        for w in ws:
+            w.release()
     return rows
 
 

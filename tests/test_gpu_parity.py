@@ -360,6 +360,29 @@ def test_gemm_tcgen05(N, K, gs, m):
         assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_AUTO), ref, f"auto {N}x{K}/{gs} m={m}")
 
 
+# Shapes with fewer tiles than SMs: the tile's K is split over several CTAs
+# whose fp32 partials are summed by the last one to finish.
+TC_SPLIT_SHAPES = [
+    (256, 4096, 128, 64),   # 1 tile, 8 splits; 128-wide groups, so splits start inside a scale box
+    (300, 3088, 16, 40),    # ragged K (48.25 k-blocks), 2 tiles x 6 splits
+    (1000, 2048, 32, 200),  # 4 tiles x 4 splits, ragged N
+    (130, 8192, 64, 17),    # one 32-column tile, 16 splits
+    (256, 1088, 64, 48),    # 17 groups per row: scales by direct loads, 2 splits
+]
+
+
+@pytest.mark.parametrize("N,K,gs,m", TC_SPLIT_SHAPES)
+def test_gemm_tcgen05_split_k(N, K, gs, m):
+    W, g = make(41, N, K, gs)
+    X = synth.activations(g, m, K)
+    ref = oracle.gemm(*W.host, gs, X)
+    y1 = run_gemm(W, X, m, mq.MLXQ_GEMM_TCGEN05)
+    assert_close(y1, ref, f"tc split {N}x{K}/{gs} m={m}")
+    # the partials are added in split order whichever CTA finishes last
+    y2 = run_gemm(W, X, m, mq.MLXQ_GEMM_TCGEN05)
+    assert np.array_equal(y1, y2)
+
+
 def test_gemm_tcgen05_integer_weights_exact():
     # s = 1, b = 0 and small-integer X: every BF16 product and fp32 partial sum is
     # an exact integer below 2^24, so the tensor-core result must equal the

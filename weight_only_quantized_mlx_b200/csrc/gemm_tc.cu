@@ -1,23 +1,32 @@
-// Tensor-core gemm for large m ("MlxInt8Weight" page, gemm: Y = X W^T).
+// Tensor-core gemm for m > 32 ("MlxInt8Weight" page, gemm: Y = X W^T).
 //
 // The page's kernel computes one output element per thread; here the
-// contraction runs on the sm_100 tensor cores instead:
+// contraction runs on the sm_100 tensor cores (tcgen05) instead.
 //
-//   CTA tile: 128 weight rows (MMA M) x BN activation rows (MMA N), full K.
-//   warp 0      TMA producer: per 64-wide k-block, the packed bytes of the
-//               128 weight rows (2-D tensor copy, no swizzle) and the BN x 64
-//               BF16 activation tile (2-D tensor copy, 128-byte swizzle).
-//   warp 1      allocates TMEM (BN fp32 columns x 128 lanes) and, from one
+//   tile: 256 weight rows (two MMA M=128 halves) x BN activation rows (MMA N),
+//         over the k-blocks of one K split (64 codes per k-block)
+//   warp 0      TMA: the BN x 64 BF16 activation tile of each k-block
+//               (128-byte swizzle, the MMA's B operand)
+//   warp 1      allocates TMEM (2 x BN fp32 columns x 128 lanes) and, from one
 //               lane, issues tcgen05.mma kind::f16 (BF16 x BF16 -> fp32),
-//               4 per k-block, committing each stage back to the producer.
-//   warps 2-9   dequantise the packed tile to BF16 straight into the MMA's
-//               A operand layout (K-major, 128-byte swizzle) - exactly the
-//               BF16 weight dequantize_to writes - then, after the last
-//               k-block, read the accumulators (tcgen05.ld) and store Y.
+//               8 per k-block, committing each stage back to the producers
+//   warp 2      TMA: packed codes of the 256 rows, and 8-group boxes of their
+//               scales and biases
+//   warps 3-10  dequantise the codes to BF16 straight into the MMA's A
+//               operand layout (K-major, 128-byte swizzle) - exactly the BF16
+//               weight dequantize_to writes
+//   warps 11-18 after a unit's last k-block, read the accumulators
+//               (tcgen05.ld) and store Y (or the unit's fp32 partial)
 //
-// The accumulator is D[w_row][x_row] (TMEM lane = weight row), so each warp's
-// stores of one output row of Y are 32 consecutive BF16 values.  All pipeline
-// waits are bounded; no cluster multicast is used.
+// When the tiles alone would leave SMs idle, each tile's K is split over
+// several CTAs: each stores its fp32 partial tile, and the last to finish
+// (a per-tile counter) adds them in split order, so the result does not
+// depend on which CTA finishes when.  The accumulator is D[w_row][x_row]
+// (TMEM lane = weight row), so a warp's stores of one output row of Y are 32
+// consecutive BF16 values.  All pipeline waits are bounded; no cluster
+// multicast is used.
+#include <mutex>
+
 #include "device_common.cuh"
 #include "kernels.h"
 #include "tensor_map.h"
@@ -47,6 +56,9 @@ struct TcParams {
     int BN, S, num_kb;
     int sg;          // k-blocks covered by one scale/bias box (8 * gs / 64)
     int sb_tma;      // 1: scales/biases by TMA boxes; 0 (rows not 16-byte multiples): direct loads
+    int ks;          // K splits per tile (1: no split)
+    float* ws;       // ks > 1: fp32 partial tiles [tiles * ks][BN][kBM]
+    unsigned int* counters;  // ks > 1: per-tile arrival counts, zero between launches
     const uint16_t* scales;
     const uint16_t* biases;
     uint32_t stage_bytes, idesc, tmem_cols;
@@ -113,9 +125,62 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
     return d;
 }
 
-// Persistent: CTA b processes tiles b, b + gridDim.x, ... (weight-row tile
-// fastest).  A tile is 256 weight rows x BN activation rows: two M=128 MMAs per
-// 16-wide k step share the activation (B) tile.  All operand bytes arrive by
+// Sum the ks fp32 partials of one tile in split order and store BF16 Y.
+// Thread et of the 256 epilogue threads takes float4 chunks (4 rows of one
+// column) et, et + 256, ...; the loads of four splits and kRedU chunks are in
+// flight together.
+constexpr int kRedU = 4;
+__device__ __forceinline__ void reduce_partials(const TcParams& p, int tile, int n0, int m0, int cols, int et) {
+    const float* base = p.ws + static_cast<int64_t>(tile) * p.ks * p.BN * kBM;
+    const int64_t part = static_cast<int64_t>(p.BN) * kBM;  // floats per partial
+    const int nchunk = cols * (kBM / 4);
+    const bool vec_store = (p.N % 4 == 0) && ((reinterpret_cast<uintptr_t>(p.Y) & 7u) == 0);
+    for (int f0 = et; f0 < nchunk; f0 += kEpilogueWarps * 32 * kRedU) {
+        float4 acc[kRedU];
+#pragma unroll
+        for (int u = 0; u < kRedU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp0 = 0; sp0 < p.ks; sp0 += 4) {
+            float4 v[4][kRedU];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int u = 0; u < kRedU; ++u) {
+                    const int f = f0 + u * kEpilogueWarps * 32;
+                    v[i][u] = (sp0 + i < p.ks && f < nchunk)
+                                  ? __ldcg(reinterpret_cast<const float4*>(base + (sp0 + i) * part) + f)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int u = 0; u < kRedU; ++u) {
+                    acc[u].x += v[i][u].x; acc[u].y += v[i][u].y;
+                    acc[u].z += v[i][u].z; acc[u].w += v[i][u].w;
+                }
+        }
+#pragma unroll
+        for (int u = 0; u < kRedU; ++u) {
+            const int f = f0 + u * kEpilogueWarps * 32;
+            if (f >= nchunk) continue;
+            const int c = f / (kBM / 4);
+            const int n = n0 + (f % (kBM / 4)) * 4;
+            uint16_t* y = p.Y + static_cast<int64_t>(m0 + c) * p.N + n;
+            const uint32_t lo = pack_bf16x2(acc[u].x, acc[u].y), hi = pack_bf16x2(acc[u].z, acc[u].w);
+            if (vec_store && n + 3 < p.N) {
+                *reinterpret_cast<uint2*>(y) = make_uint2(lo, hi);
+            } else {
+                const uint16_t h[4] = {static_cast<uint16_t>(lo), static_cast<uint16_t>(lo >> 16),
+                                       static_cast<uint16_t>(hi), static_cast<uint16_t>(hi >> 16)};
+                for (int i = 0; i < 4 && n + i < p.N; ++i) y[i] = h[i];
+            }
+        }
+    }
+}
+
+// Persistent: CTA b processes units b, b + gridDim.x, ... (a unit is one K
+// split of one tile, weight-row tile fastest).  A tile is 256 weight rows x
+// BN activation rows: two M=128 MMAs per 16-wide k step share the activation
+// (B) tile.  All operand bytes arrive by
 // TMA: the activation tile into the (A, X) stage ring, the packed codes into
 // their own ring, and the scales/biases as 8-group boxes into a third ring;
 // the dequant warps read only shared memory.  The two fp32 accumulators fill
@@ -133,8 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tiles_n = (p.N + kBM - 1) / kBM;
     const int tiles_m = (p.m + p.BN - 1) / p.BN;
     const int num_tiles = tiles_n * tiles_m;
-    const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    const int sb_per_tile = (p.num_kb + p.sg - 1) / p.sg;
+    const int num_units = num_tiles * p.ks;
+    const int my_units = blockIdx.x < num_units ? (num_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
     // shared memory: S (A, X) stages | kSP packed slots | kSSB (scales, biases) slots | barriers
     const uint32_t sbase = smem_u32(smem);
@@ -150,15 +215,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* acc_full = sbempty + kSSB;
     uint64_t* acc_empty = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+    uint32_t* last_flag = tmem_slot + 1;  // epilogue: this CTA completed the tile
     auto A_of = [&](int s) { return sbase + static_cast<uint32_t>(s) * p.stage_bytes; };
     auto X_of = [&](int s) { return A_of(s) + kStageA; };
     auto P_of = [&](int s) { return p_base + static_cast<uint32_t>(s) * kStageP; };
     auto SC_of = [&](int s) { return sb_base + static_cast<uint32_t>(s) * 2u * kStageSB; };
     auto BI_of = [&](int s) { return SC_of(s) + kStageSB; };
-    auto tile_nm = [&](int t, int& n0, int& m0) {
-        const int tile = blockIdx.x + t * gridDim.x;
+    // Work unit t of this CTA: a tile (weight-row tile fastest) and the
+    // k-blocks [kb0, kb1) of its K split.
+    auto unit_of = [&](int t, int& tile, int& split, int& n0, int& m0, int& kb0, int& kb1) {
+        const int u = blockIdx.x + t * gridDim.x;
+        tile = u % num_tiles;
+        split = u / num_tiles;
         n0 = (tile % tiles_n) * kBM;
         m0 = (tile / tiles_n) * p.BN;
+        kb0 = static_cast<int>(static_cast<int64_t>(split) * p.num_kb / p.ks);
+        kb1 = static_cast<int>(static_cast<int64_t>(split + 1) * p.num_kb / p.ks);
     };
 
     pdl_launch_dependents();
@@ -196,10 +268,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = policy_evict_last();  // each activation tile serves every weight tile
             bool ok = true;
             int it = 0;
-            for (int t = 0; t < my_tiles; ++t) {
-                int n0, m0;
-                tile_nm(t, n0, m0);
-                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+            for (int t = 0; t < my_units; ++t) {
+                int tile, split, n0, m0, kb0, kb1;
+                unit_of(t, tile, split, n0, m0, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     if (it >= S && ok) ok = mbar_wait(smem_u32(&empty[s]), ((it / S) - 1) & 1, p.status);
                     mbar_arrive_expect_tx(smem_u32(&full[s]), stage_x);
@@ -218,11 +290,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = policy_evict_last();  // each weight tile serves every activation tile
             bool ok = true;
             int it = 0, sbi = 0;
-            for (int t = 0; t < my_tiles; ++t) {
-                int n0, m0;
-                tile_nm(t, n0, m0);
-                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-                    if (p.sb_tma && kb % p.sg == 0) {  // a new scale/bias box for the next sg k-blocks
+            for (int t = 0; t < my_units; ++t) {
+                int tile, split, n0, m0, kb0, kb1;
+                unit_of(t, tile, split, n0, m0, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    if (p.sb_tma && (kb == kb0 || kb % p.sg == 0)) {  // the scale/bias box holding kb
                         const int ss = sbi % kSSB;
                         if (sbi >= kSSB && ok) ok = mbar_wait(smem_u32(&sbempty[ss]), ((sbi / kSSB) - 1) & 1, p.status);
                         mbar_arrive_expect_tx(smem_u32(&sbfull[ss]), 2u * kStageSB);
@@ -243,12 +315,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             bool ok = true;
             int it = 0;
-            for (int t = 0; t < my_tiles; ++t) {
-                // the epilogue must have drained the accumulators (previous tile)
+            for (int t = 0; t < my_units; ++t) {
+                int tile, split, n0, m0, kb0, kb1;
+                unit_of(t, tile, split, n0, m0, kb0, kb1);
+                // the epilogue must have drained the accumulators (previous unit)
                 if (t >= 1 && ok) ok = mbar_wait(smem_u32(acc_empty), (t - 1) & 1, p.status);
                 tc_fence_after();
                 const uint32_t d0 = tmem_base, d1 = tmem_base + p.tmem_cols;
-                for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     if (ok) ok = mbar_wait(smem_u32(&full[s]), (it / S) & 1, p.status);
                     tc_fence_after();
@@ -258,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         // advance 16 BF16 (32 bytes) along K inside the swizzled rows
-                        const uint32_t acc = (kb | kk) != 0;
+                        const uint32_t acc = (kb != kb0 || kk != 0) ? 1u : 0u;
                         umma_bf16(d0, a0 + 2u * kk, bd + 2u * kk, p.idesc, acc);
                         umma_bf16(d1, a1 + 2u * kk, bd + 2u * kk, p.idesc, acc);
                     }
@@ -276,30 +350,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         const float2 m2 = make_float2(-kMagic, -kMagic);
         int it = 0, sbi = 0;
-        for (int t = 0; t < my_tiles; ++t) {
-            for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        for (int t = 0; t < my_units; ++t) {
+            int tile, split, n0, m0, kb0, kb1;
+            unit_of(t, tile, split, n0, m0, kb0, kb1);
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int ss = sbi % kSSB;
-                if (p.sb_tma && kb % p.sg == 0 && ok) ok = mbar_wait(smem_u32(&sbfull[ss]), (sbi / kSSB) & 1, p.status);
+                if (p.sb_tma && (kb == kb0 || kb % p.sg == 0) && ok)
+                    ok = mbar_wait(smem_u32(&sbfull[ss]), (sbi / kSSB) & 1, p.status);
                 const int sp = it % kSP;
                 if (ok) ok = mbar_wait(smem_u32(&pfull[sp]), (it / kSP) & 1, p.status);
-                // this thread's codes and the scale/bias of their group, for 4 rows
+                // this thread's codes and the scale/bias of their group, for its 4 rows
                 const int gl = ((kb % p.sg) * kBK + chunk * 16) / p.gs;  // group within the box
                 uint4 wq[4];
                 float2 s2[4], b2[4];
-                int n0 = 0, m0 = 0;
-                if (!p.sb_tma) tile_nm(t, n0, m0);
                 const int k0 = kb * kBK + chunk * 16;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int row = rbase + 64 * i;
-                    wq[i] = lds128(P_of(sp) + static_cast<uint32_t>(row * kBK + chunk * 16));
+                    const int drow = rbase + 64 * i;
+                    wq[i] = lds128(P_of(sp) + static_cast<uint32_t>(drow * kBK + chunk * 16));
                     float sv = 0.f, bv = 0.f;
                     if (p.sb_tma) {
-                        const uint32_t so = static_cast<uint32_t>(row * kSbGroups + gl) * 2u;
+                        const uint32_t so = static_cast<uint32_t>(drow * kSbGroups + gl) * 2u;
                         sv = bf16_bits_to_f32(lds16(SC_of(ss) + so));
                         bv = bf16_bits_to_f32(lds16(BI_of(ss) + so));
-                    } else if (n0 + row < p.N && k0 < p.K) {
-                        const int64_t gi = static_cast<int64_t>(n0 + row) * p.G + k0 / p.gs;
+                    } else if (n0 + drow < p.N && k0 < p.K) {
+                        const int64_t gi = static_cast<int64_t>(n0 + drow) * p.G + k0 / p.gs;
                         sv = bf16_bits_to_f32(__ldg(p.scales + gi));
                         bv = bf16_bits_to_f32(__ldg(p.biases + gi));
                     }
@@ -308,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&pempty[sp]));  // packed slot read
-                if (p.sb_tma && (kb % p.sg == p.sg - 1 || kb == p.num_kb - 1)) {
+                if (p.sb_tma && (kb % p.sg == p.sg - 1 || kb == kb1 - 1)) {
                     if (lane == 0) mbar_arrive(smem_u32(&sbempty[ss]));  // last use of this box
                     ++sbi;
                 }
@@ -317,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (it >= S && ok) ok = mbar_wait(smem_u32(&empty[s]), ((it / S) - 1) & 1, p.status);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int row = rbase + 64 * i;  // 0..255: half row >> 7
+                    const int drow = rbase + 64 * i;  // 0..255: half drow >> 7
                     const uint32_t words[4] = {wq[i].x, wq[i].y, wq[i].z, wq[i].w};
                     uint32_t o[8];
 #pragma unroll
@@ -332,8 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     // logical 16-byte chunks 2*chunk and 2*chunk+1 of this 128-byte row,
                     // placed by the 128-byte swizzle (chunk index ^ row % 8)
-                    const uint32_t rowa = A_of(s) + static_cast<uint32_t>(row) * 128u;
-                    const uint32_t sw = static_cast<uint32_t>(row & 7);
+                    const uint32_t rowa = A_of(s) + static_cast<uint32_t>(drow) * 128u;
+                    const uint32_t sw = static_cast<uint32_t>(drow & 7);
                     sts128(rowa + (((2u * chunk) ^ sw) << 4), o[0], o[1], o[2], o[3]);
                     sts128(rowa + (((2u * chunk + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
                 }
@@ -350,32 +425,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int half = ew >> 2;              // accumulator half
         const int row = half * kHM + q * 32 + lane;
         bool ok = true;
-        for (int t = 0; t < my_tiles; ++t) {
-            int n0, m0;
-            tile_nm(t, n0, m0);
+        for (int t = 0; t < my_units; ++t) {
+            int tile, split, n0, m0, kb0, kb1;
+            unit_of(t, tile, split, n0, m0, kb0, kb1);
             if (ok) ok = mbar_wait(smem_u32(acc_full), t & 1, p.status);
             tc_fence_after();
             const uint32_t d = tmem_base + static_cast<uint32_t>(half) * p.tmem_cols +
                                (static_cast<uint32_t>(q * 32) << 16);
             const int n = n0 + row;
             const int cols = p.m - m0 < p.BN ? p.m - m0 : p.BN;
+            if (p.ks == 1) {
+                for (int c0 = 0; c0 < cols; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(d + static_cast<uint32_t>(c0), r);
+                    tmem_ld_wait();
+                    if (n < p.N) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            if (c0 + j < cols) {
+                                const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
+                                p.Y[static_cast<int64_t>(m0 + c0 + j) * p.N + n] = *reinterpret_cast<const uint16_t*>(&v);
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(acc_empty));
+                continue;
+            }
+            // K split: store this split's fp32 partial ([column][row], so a
+            // warp's stores are 128 contiguous bytes), free the accumulators,
+            // and let the tile's last unit to finish add the ks partials in
+            // split order (the same order whichever unit is last).
+            float* part = p.ws + (static_cast<int64_t>(tile) * p.ks + split) * p.BN * kBM;
             for (int c0 = 0; c0 < cols; c0 += 16) {
                 uint32_t r[16];
                 tmem_ld16(d + static_cast<uint32_t>(c0), r);
                 tmem_ld_wait();
-                if (n < p.N) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        if (c0 + j < cols) {
-                            const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[j]));
-                            p.Y[static_cast<int64_t>(m0 + c0 + j) * p.N + n] = *reinterpret_cast<const uint16_t*>(&v);
-                        }
-                    }
-                }
+                for (int j = 0; j < 16; ++j)
+                    if (c0 + j < cols) __stcg(part + static_cast<int64_t>(c0 + j) * kBM + row, __uint_as_float(r[j]));
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(acc_empty));
+            __threadfence();  // this thread's partial is visible before the tile's count moves
+            named_bar_sync(1, kEpilogueWarps * 32);
+            if (ew == 0 && lane == 0) {
+                const unsigned int prev = atomicAdd(p.counters + tile, 1u);
+                const bool last = prev == static_cast<unsigned int>(p.ks - 1);
+                if (last) p.counters[tile] = 0u;  // zero again for the next launch
+                *reinterpret_cast<volatile uint32_t*>(last_flag) = last ? 1u : 0u;
+            }
+            named_bar_sync(1, kEpilogueWarps * 32);
+            const bool last = *reinterpret_cast<volatile uint32_t*>(last_flag) != 0u;
+            if (last) {
+                __threadfence();
+                reduce_partials(p, tile, n0, m0, cols, ew * 32 + lane);
+            }
+            named_bar_sync(1, kEpilogueWarps * 32);  // the flag is read before the next unit rewrites it
         }
     }
     tc_fence_before();
@@ -390,6 +499,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 int pick_bn(int64_t m) {
     int64_t bn = (m + 31) / 32 * 32;
     return static_cast<int>(bn > 256 ? 256 : bn);
+}
+
+// The library's own stream-ordered pool for split-K partials, one per device:
+// it keeps its memory between calls (the device's default pool hands memory
+// back at every synchronisation, and mapping it again costs more than the
+// kernel).
+cudaError_t workspace_pool(int device, cudaMemPool_t* out) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64];
+    static bool made[64];
+    if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!made[device]) {
+        cudaMemPoolProps props{};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = device;
+        cudaError_t e = cudaMemPoolCreate(&pools[device], &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = ~0ull;
+        e = cudaMemPoolSetAttribute(pools[device], cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) return e;
+        made[device] = true;
+    }
+    *out = pools[device];
+    return cudaSuccess;
+}
+
+constexpr int kMinKbPerSplit = 8;  // 512 codes: a split shorter than this is mostly pipeline fill
+
+// K splits per tile: only when the tiles alone leave SMs idle; as many as
+// keep every split in one wave (units <= SMs) and >= kMinKbPerSplit long.
+int pick_ks(int64_t tiles, int num_kb, int sm_count) {
+    if (tiles >= sm_count) return 1;
+    int64_t ks = sm_count / tiles;
+    const int64_t by_k = num_kb / kMinKbPerSplit;
+    if (ks > by_k) ks = by_k;
+    return ks < 1 ? 1 : static_cast<int>(ks);
 }
 
 }  // namespace
@@ -420,6 +568,9 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
     p.num_kb = static_cast<int>((w.K + kBK - 1) / kBK);
     p.sg = static_cast<int>(kSbGroups * w.gs / kBK);
     p.sb_tma = (w.G % 8 == 0) ? 1 : 0;
+    const int64_t tiles = ((w.N + kBM - 1) / kBM) * ((m + p.BN - 1) / p.BN);
+    if (tiles > (1ll << 30)) return cudaErrorInvalidValue;
+    p.ks = pick_ks(tiles, p.num_kb, dev.sm_count);
     p.scales = w.scales;
     p.biases = w.biases;
     p.stage_bytes = kStageA + static_cast<uint32_t>(p.BN) * 128u;
@@ -451,12 +602,31 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
     static std::atomic<int> configured[64];
     cudaError_t e = ensure_dynamic_smem(k_gemm_tc, smem, configured);
     if (e != cudaSuccess) return e;
-    const int64_t tiles = ((w.N + kBM - 1) / kBM) * ((m + p.BN - 1) / p.BN);
-    if (tiles > (1ll << 31) - 1) return cudaErrorInvalidValue;
-    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-    e = launch_pdl(k_gemm_tc, dim3(grid), dim3(kThreads), smem, stream, tm_x, wm.packed, wm.scales, wm.biases, p);
+    const int64_t units = tiles * p.ks;
+    const int grid = static_cast<int>(units < dev.sm_count ? units : dev.sm_count);
+    if (p.ks == 1) {
+        e = launch_pdl(k_gemm_tc, dim3(grid), dim3(kThreads), smem, stream, tm_x, wm.packed, wm.scales, wm.biases, p);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
+    // K split: the fp32 partials and the per-tile counters come from the
+    // stream-ordered pool (so the call also works under graph capture)
+    const size_t part_bytes = static_cast<size_t>(units) * p.BN * kBM * sizeof(float);
+    const size_t bytes = part_bytes + static_cast<size_t>(tiles) * sizeof(unsigned int);
+    cudaMemPool_t pool;
+    e = workspace_pool(dev.device, &pool);
     if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    void* ws = nullptr;
+    e = cudaMallocFromPoolAsync(&ws, bytes, pool, stream);
+    if (e != cudaSuccess) return e;
+    p.ws = static_cast<float*>(ws);
+    p.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + part_bytes);
+    e = cudaMemsetAsync(p.counters, 0, static_cast<size_t>(tiles) * sizeof(unsigned int), stream);
+    if (e == cudaSuccess)
+        e = launch_pdl(k_gemm_tc, dim3(grid), dim3(kThreads), smem, stream, tm_x, wm.packed, wm.scales, wm.biases, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    const cudaError_t ef = cudaFreeAsync(ws, stream);
+    return e != cudaSuccess ? e : ef;
 }
 
 }  // namespace mlxq
