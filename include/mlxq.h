@@ -125,16 +125,37 @@ MLXQ_API int mlxq_gemv_silu_gate_resid(const mlxq_weight* w, const void* gate, c
  * a no-op.  The kernel is chosen from m: weight-streaming kernels for small m
  * (every weight byte read once, dequantised in registers) or the tcgen05
  * tensor-core kernel for larger m (weight tiles dequantised to BF16 in shared
- * memory, fp32 accumulators in TMEM).
+ * memory, fp32 accumulators in TMEM).  When m leaves SMs idle, the
+ * tensor-core kernel splits K over CTAs; their fp32 partials live in a
+ * stream-ordered memory pool owned by the library (allocated and freed on
+ * `stream`, so the call can be captured in a CUDA graph).
  */
 MLXQ_API int mlxq_gemm(const mlxq_weight* w, const void* x, void* y, uint32_t m, uint64_t stream);
+
+/* Size of the scratch buffer compiled into the library for mlxq_gemm_noalloc:
+ * enough for every K split on a GPU with up to 148 SMs (at most one CTA per SM
+ * per split tile, 256 x 256 fp32 partials each) plus the tile counters. */
+#define MLXQ_STATIC_SCRATCH_BYTES (40u << 20)
+
+/*
+ * mlxq_gemm_noalloc (page: MlxInt8Weight::gemm, kernel mlx_int8_gemm).
+ * mlxq_gemm that allocates no device memory: same arguments, layout, kernel
+ * choice and results (bit for bit).  Where mlxq_gemm takes the K-split
+ * partials from its memory pool, this call uses the library's static scratch
+ * buffer (MLXQ_STATIC_SCRATCH_BYTES, a device array that exists from the
+ * moment the library's device code loads).  A call whose split would need
+ * more returns MLXQ_ERR_UNSUPPORTED and launches nothing.  The buffer is one
+ * per device and shared by every call, so calls that split K must not run at
+ * the same time: issue them on one stream, or order them with events.
+ */
+MLXQ_API int mlxq_gemm_noalloc(const mlxq_weight* w, const void* x, void* y, uint32_t m, uint64_t stream);
 
 /* Kernel selection for mlxq_gemm_with (tests and benchmarks pin a path). */
 enum {
     MLXQ_GEMM_AUTO = 0,        /* what mlxq_gemm picks */
     MLXQ_GEMM_ROWS = 1,        /* m independent passes of the gemv kernel */
     MLXQ_GEMM_SMALLM = 2,      /* weight-streaming kernel, products on the tensor pipe
-                                  (mma.sync fragments), m <= 8 */
+                                  (mma.sync fragments), m <= 32 */
     MLXQ_GEMM_TCGEN05 = 3,     /* tcgen05 tensor-core kernel (TMEM accumulators) */
     MLXQ_GEMM_SMALLM_FFMA = 4  /* weight-streaming kernel on the fp32 pipes, m <= 32 */
 };

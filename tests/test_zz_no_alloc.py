@@ -1,0 +1,114 @@
+"""mlxq_gemm_noalloc: the gemm entry point that allocates no device memory.
+
+Its K-split partials live in the library's static scratch buffer instead of
+the stream-ordered pool.  Checked here: results equal mlxq_gemm bit for bit
+and the oracle within the gemm tolerance; two calls in a row (no
+synchronisation between them, so the second starts from the counters the
+first left behind) both stay exact; and a CUDA graph holding two calls
+replays correctly, which it could not do if the call allocated.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_only_quantized_mlx_b200 as mq
+from _helpers import Guarded, assert_close, dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "the -m gpu tests need a CUDA device"
+    yield
+    mq.mlxq_device_status()
+
+
+def weight(seed, N, K, gs):
+    g = synth.rng(seed)
+    host = synth.weight(g, N, K, gs)
+    t = tuple(dev(a) for a in host)
+    return host, t, mq.weight_view(*t, gs), g
+
+
+def call(fn, w, X, m, N):
+    Y = Guarded(m * N)
+    fn(w, X, Y.data_ptr(), m)
+    torch.cuda.synchronize()
+    Y.check_guards()
+    return Y.value_bits().reshape(m, N)
+
+
+# (N, K, gs, m): K split over CTAs (first three), whole tiles, and the
+# weight-streaming kernel (m <= 32, no scratch at all)
+SHAPES = [
+    (512, 4096, 64, 64),
+    (1000, 2048, 32, 200),
+    (256, 4096, 128, 17 + 32),
+    (256, 960, 64, 100),
+    (300, 2048, 64, 24),
+]
+
+
+@pytest.mark.parametrize("N,K,gs,m", SHAPES)
+def test_noalloc_matches_gemm_and_oracle(N, K, gs, m):
+    host, keep, w, g = weight(70 + m, N, K, gs)
+    X_bits = synth.activations(g, m, K)
+    X = dev(X_bits)
+    y_na = call(mq.mlxq_gemm_noalloc, w, X, m, N)
+    y_ref = call(mq.mlxq_gemm, w, X, m, N)
+    assert np.array_equal(y_na, y_ref)
+    assert_close(y_na, oracle.gemm(*host, gs, X_bits), f"noalloc {N}x{K}/{gs} m={m}")
+
+
+def test_noalloc_two_calls_in_a_row():
+    # different shapes, back to back on one stream with no synchronisation
+    ha, keep_a, wa, ga = weight(80, 512, 4096, 64)  # keep_*: the device arrays the views point at
+    hb, keep_b, wb, gb = weight(81, 1000, 2048, 32)
+    Xa_bits, Xb_bits = synth.activations(ga, 64, 4096), synth.activations(gb, 200, 2048)
+    Xa, Xb = dev(Xa_bits), dev(Xb_bits)
+    Ya, Yb = Guarded(64 * 512), Guarded(200 * 1000)
+    mq.mlxq_gemm_noalloc(wa, Xa, Ya.data_ptr(), 64)
+    mq.mlxq_gemm_noalloc(wb, Xb, Yb.data_ptr(), 200)
+    mq.mlxq_gemm_noalloc(wa, Xa, Ya.data_ptr(), 64)  # the first shape again, after the second
+    torch.cuda.synchronize()
+    Ya.check_guards()
+    Yb.check_guards()
+    ya, yb = Ya.value_bits().reshape(64, 512), Yb.value_bits().reshape(200, 1000)
+    assert np.array_equal(ya, call(mq.mlxq_gemm, wa, Xa, 64, 512))
+    assert np.array_equal(yb, call(mq.mlxq_gemm, wb, Xb, 200, 1000))
+    assert_close(ya, oracle.gemm(*ha, 64, Xa_bits), "noalloc, first call")
+    assert_close(yb, oracle.gemm(*hb, 32, Xb_bits), "noalloc, second call")
+
+
+def test_noalloc_in_a_cuda_graph():
+    host, keep, w, g = weight(82, 512, 4096, 64)
+    m = 96
+    X_bits = synth.activations(g, m, 4096)
+    X = dev(X_bits)
+    Y1 = torch.zeros(m * 512, dtype=torch.int16, device="cuda")
+    Y2 = torch.zeros(m * 512, dtype=torch.int16, device="cuda")
+    mq.mlxq_gemm_noalloc(w, X, Y1, m)  # warm-up outside capture (module load, tensor maps)
+    torch.cuda.synchronize()
+    Y1.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        mq.mlxq_gemm_noalloc(w, X, Y1, m)
+        mq.mlxq_gemm_noalloc(w, X, Y2, m)
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    y_ref = call(mq.mlxq_gemm, w, X, m, 512)
+    assert np.array_equal(Y1.cpu().numpy().view(np.uint16).reshape(m, 512), y_ref)
+    assert np.array_equal(Y2.cpu().numpy().view(np.uint16).reshape(m, 512), y_ref)
+    del graph
+
+
+def test_noalloc_scratch_covers_every_split_on_this_gpu():
+    # the largest split the kernel makes: one CTA per SM, 256 x 256 fp32 each
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert 4096 + sms * 256 * 256 * 4 <= mq.MLXQ_STATIC_SCRATCH_BYTES

@@ -37,7 +37,7 @@ MLXQ_GEMM_TCGEN05 = 3
 MLXQ_GEMM_SMALLM_FFMA = 4
 
 EXPORTS = ("mlxq_load", "mlxq_dequant", "mlxq_gemv", "mlxq_gemv_silu_gate",
-           "mlxq_gemv_silu_gate_resid", "mlxq_gemm", "mlxq_gemm_with", "mlxq_release",
+           "mlxq_gemv_silu_gate_resid", "mlxq_gemm", "mlxq_gemm_with", "mlxq_gemm_noalloc", "mlxq_release",
            "mlxq_last_error", "mlxq_device_status")
 
 
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "mlxq_gemv_silu_gate_resid": [W, vp, vp, vp, vp, u64],
             "mlxq_gemm": [W, vp, vp, u32, u64],
             "mlxq_gemm_with": [W, vp, vp, u32, i32, u64],
+            "mlxq_gemm_noalloc": [W, vp, vp, u32, u64],
             "mlxq_release": [W],
             "mlxq_last_error": [],
             "mlxq_device_status": [],
@@ -144,6 +145,13 @@ def mlxq_gemm(w: mlxq_weight, x, y, m: int, stream=None) -> None:
 
 def mlxq_gemm_with(w: mlxq_weight, x, y, m: int, kernel: int, stream=None) -> None:
     _check(lib().mlxq_gemm_with(ctypes.byref(w), _ptr(x), _ptr(y), m, kernel, _stream(stream)))
+
+
+def mlxq_gemm_noalloc(w: mlxq_weight, x, y, m: int, stream=None) -> None:
+    _check(lib().mlxq_gemm_noalloc(ctypes.byref(w), _ptr(x), _ptr(y), m, _stream(stream)))
+
+
+MLXQ_STATIC_SCRATCH_BYTES = 40 << 20
 
 
 def mlxq_device_status() -> None:

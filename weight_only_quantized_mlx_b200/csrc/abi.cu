@@ -525,7 +525,10 @@ int mlxq_gemv_silu_gate_resid(const mlxq_weight* w, const void* gate, const void
 // Kernel choice by m: the weight-streaming kernels read every weight byte
 // once and are HBM-bound while the per-byte work fits the SM; beyond
 // kStreamMmaMaxM rows the tcgen05 kernel takes over.
-int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kernel, uint64_t stream) {
+namespace {
+
+int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kernel, uint64_t stream,
+              TcScratch scratch) {
     WeightView v;
     int rc = check_weight(w, v);
     if (rc) return rc;
@@ -574,12 +577,26 @@ int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32_t m, int
                 return fail(MLXQ_ERR_UNSUPPORTED, "tensor-core kernel cannot take m=%lld, N=%lld, K=%lld, group_size=%lld",
                             static_cast<long long>(M), static_cast<long long>(v.N), static_cast<long long>(v.K),
                             static_cast<long long>(v.gs));
-            return launch_status(launch_gemm_tc(v, x, y, M, s), "tcgen05 gemm launch");
+            if (scratch == TC_SCRATCH_STATIC && gemm_tc_scratch_bytes(v, M) > kStaticScratchBytes)
+                return fail(MLXQ_ERR_UNSUPPORTED, "K split of m=%lld, N=%lld needs %zu bytes of scratch; the static buffer holds %zu",
+                            static_cast<long long>(M), static_cast<long long>(v.N), gemm_tc_scratch_bytes(v, M),
+                            kStaticScratchBytes);
+            return launch_status(launch_gemm_tc(v, x, y, M, s, scratch), "tcgen05 gemm launch");
     }
 }
 
+}  // namespace
+
+int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kernel, uint64_t stream) {
+    return gemm_impl(w, x, y, m, kernel, stream, TC_SCRATCH_POOL);
+}
+
 int mlxq_gemm(const mlxq_weight* w, const void* x, void* y, uint32_t m, uint64_t stream) {
-    return mlxq_gemm_with(w, x, y, m, MLXQ_GEMM_AUTO, stream);
+    return gemm_impl(w, x, y, m, MLXQ_GEMM_AUTO, stream, TC_SCRATCH_POOL);
+}
+
+int mlxq_gemm_noalloc(const mlxq_weight* w, const void* x, void* y, uint32_t m, uint64_t stream) {
+    return gemm_impl(w, x, y, m, MLXQ_GEMM_AUTO, stream, TC_SCRATCH_STATIC);
 }
 
 int mlxq_device_status(void) {

@@ -32,6 +32,11 @@
 #include "tensor_map.h"
 
 namespace mlxq {
+
+// Scratch of mlxq_gemm_noalloc, compiled into the library (zero when the
+// module loads): per-tile counters, then the fp32 partials.  Every split
+// gemm leaves the counters it used at zero, so calls need no reset.
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 namespace {
 
 constexpr int kBM = 256;                // weight rows per tile: two MMA M=128 halves
@@ -530,6 +535,23 @@ cudaError_t workspace_pool(int device, cudaMemPool_t* out) {
 
 constexpr int kMinKbPerSplit = 8;  // 512 codes: a split shorter than this is mostly pipeline fill
 
+constexpr size_t kCounterBytes = 4096;  // room for 1024 tile counters
+
+cudaError_t static_scratch_base(int device, unsigned char** out) {
+    static std::mutex mu;
+    static unsigned char* base[64];
+    if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (base[device] == nullptr) {
+        void* a = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&a, g_static_scratch);
+        if (e != cudaSuccess) return e;
+        base[device] = static_cast<unsigned char*>(a);
+    }
+    *out = base[device];
+    return cudaSuccess;
+}
+
 // K splits per tile: only when the tiles alone leave SMs idle; as many as
 // keep every split in one wave (units <= SMs) and >= kMinKbPerSplit long.
 int pick_ks(int64_t tiles, int num_kb, int sm_count) {
@@ -555,7 +577,18 @@ bool gemm_tc_supported(const WeightView& w, int64_t m, const void* X, const void
     return tensor_maps_available();
 }
 
-cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream) {
+size_t gemm_tc_scratch_bytes(const WeightView& w, int64_t m) {
+    const DeviceInfo& dev = device_info();
+    const int bn = pick_bn(m);
+    const int num_kb = static_cast<int>((w.K + kBK - 1) / kBK);
+    const int64_t tiles = ((w.N + kBM - 1) / kBM) * ((m + bn - 1) / bn);
+    const int ks = pick_ks(tiles, num_kb, dev.sm_count);
+    if (ks == 1) return 0;
+    return kCounterBytes + static_cast<size_t>(tiles) * ks * bn * kBM * sizeof(float);
+}
+
+cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream,
+                           TcScratch scratch) {
     const DeviceInfo& dev = device_info();
     TcParams p{};
     p.Y = static_cast<uint16_t*>(Y);
@@ -609,9 +642,22 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
+    const size_t part_bytes = static_cast<size_t>(units) * p.BN * kBM * sizeof(float);
+    if (tiles * sizeof(unsigned int) > kCounterBytes) return cudaErrorInvalidValue;
+    if (scratch == TC_SCRATCH_STATIC) {
+        // the library's static buffer: counters already zero, nothing allocated
+        if (kCounterBytes + part_bytes > kStaticScratchBytes) return cudaErrorMemoryAllocation;
+        unsigned char* base = nullptr;
+        e = static_scratch_base(dev.device, &base);
+        if (e != cudaSuccess) return e;
+        p.counters = reinterpret_cast<unsigned int*>(base);
+        p.ws = reinterpret_cast<float*>(base + kCounterBytes);
+        e = launch_pdl(k_gemm_tc, dim3(grid), dim3(kThreads), smem, stream, tm_x, wm.packed, wm.scales, wm.biases, p);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
     // K split: the fp32 partials and the per-tile counters come from the
     // stream-ordered pool (so the call also works under graph capture)
-    const size_t part_bytes = static_cast<size_t>(units) * p.BN * kBM * sizeof(float);
     const size_t bytes = part_bytes + static_cast<size_t>(tiles) * sizeof(unsigned int);
     cudaMemPool_t pool;
     e = workspace_pool(dev.device, &pool);

@@ -3,6 +3,8 @@
 // shapes and alignment.  Each returns the launch status (cudaGetLastError).
 #pragma once
 
+#include "mlxq.h"
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -91,7 +93,13 @@ cudaError_t launch_gemm_smallm(const WeightView& w, const void* X, void* Y, int6
 
 // tcgen05 tensor-core gemm.
 bool gemm_tc_supported(const WeightView& w, int64_t m, const void* X, const void* Y);
-cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t m,
-                           cudaStream_t stream);
+// Where the K-split partials of the tcgen05 gemm live: the library's
+// stream-ordered pool, or the static buffer of mlxq_gemm_noalloc.
+enum TcScratch { TC_SCRATCH_POOL = 0, TC_SCRATCH_STATIC = 1 };
+constexpr size_t kStaticScratchBytes = MLXQ_STATIC_SCRATCH_BYTES;
+// Scratch bytes a tcgen05 gemm of this shape needs (0: no K split).
+size_t gemm_tc_scratch_bytes(const WeightView& w, int64_t m);
+cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream,
+                           TcScratch scratch = TC_SCRATCH_POOL);
 
 }  // namespace mlxq
