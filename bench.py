@@ -358,6 +358,30 @@ def measure_rows(mq, torch, synth, dev, stream, dec_weights, peaks, args):
         for w in ws:
             w.release()
 
+    # the same MLP with gate and up loaded as one [2F, D] weight: two launches
+    # per layer (gemv into [gate | up], then silu_gate_resid)
+    mlps = []
+    for j in range(4):
+        g = synth.rng(1000 + j)
+        pg, sg, bg = synth.weight(g, F, D, gs)
+        pu, su, bu = synth.weight(g, F, D, gs)
+        wgu = upload_weight(mq, np.concatenate([pg, pu]), np.concatenate([sg, su]), np.concatenate([bg, bu]), gs)
+        mlps.append((wgu, upload_weight(mq, *synth.weight(g, D, F, gs), gs)))
+    gu = torch.empty(2 * F, dtype=torch.bfloat16, device=dev)
+
+    def mlp2():
+        for wgu, wd in mlps:
+            mq.mlxq_gemv(wgu.handle, x, gu, stream)
+            mq.mlxq_gemv_silu_gate_resid(wd.handle, gu[:F], gu[F:], xr, y, stream)
+    ms = time_region(mlp2, steps, warm, stream, 1)
+    us = ms * 1e3 / len(mlps)
+    gbs = b / (us * 1e-6) / 1e9
+    rows["fused_mlp_decode_concat"] = {"value": round(gbs, 1), "unit": "GB/s", "us_per_mlp": round(us, 2),
+                                       "frac_hbm": round(gbs / hbm, 4), "bytes_per_mlp": b, "launches_per_mlp": 2}
+    for ws in mlps:
+        for w in ws:
+            w.release()
+
     # small-m batched decode: (N, K) in {(28672, 8192), (8192, 28672)}, gs = 64
     for (N, K) in ((28672, 8192), (8192, 28672)):
         w = upload_weight(mq, *synth.weight(synth.rng(3000 + N), N, K, 64), 64)

@@ -246,6 +246,34 @@ def test_fused_mlp_chain():
     assert_close(host_bits(y), ref_unfused, "down (unfused reference)", elementwise=False)
 
 
+def test_fused_mlp_chain_concatenated_gate_up():
+    """Gate and up loaded as one [2F, D] weight: one gemv gives [gate | up],
+    and silu_gate_resid reads the two halves in place.  Every row is computed
+    exactly as in the three-launch chain, so the output is identical."""
+    D, F, gs = 4096, 14336, 64
+    Wg, g = make(30, F, D, gs)
+    Wu, _ = make(31, F, D, gs)
+    Wd, _ = make(32, D, F, gs)
+    Wgu = DevWeight(*(np.concatenate([a, b]) for a, b in zip(Wg.host, Wu.host)), gs)
+    x = synth.activations(g, D)
+    xr = synth.activations(g, D)
+    xd, xrd = dev(x), dev(xr)
+    gu = torch.empty(2 * F, dtype=torch.bfloat16, device="cuda")
+    mq.mlxq_gemv(Wgu.w, xd, gu)
+    y2 = torch.empty(D, dtype=torch.bfloat16, device="cuda")
+    mq.mlxq_gemv_silu_gate_resid(Wd.w, gu[:F], gu[F:], xrd, y2)
+    gate = torch.empty(F, dtype=torch.bfloat16, device="cuda")
+    up = torch.empty(F, dtype=torch.bfloat16, device="cuda")
+    mq.mlxq_gemv(Wg.w, xd, gate)
+    mq.mlxq_gemv(Wu.w, xd, up)
+    y3 = torch.empty(D, dtype=torch.bfloat16, device="cuda")
+    mq.mlxq_gemv_silu_gate_resid(Wd.w, gate, up, xrd, y3)
+    gub = host_bits(gu)
+    assert np.array_equal(gub[:F], host_bits(gate)) and np.array_equal(gub[F:], host_bits(up))
+    assert np.array_equal(host_bits(y2), host_bits(y3))
+    assert_close(host_bits(y2), oracle.silu_gate_resid(*Wd.host, gs, gub[:F], gub[F:], xr), "down after concatenated gate/up")
+
+
 # ---------------------------------------------------------------- gemm
 def run_gemm(W, X_bits, m, kernel=mq.MLXQ_GEMM_AUTO):
     X = dev(X_bits)
