@@ -166,6 +166,24 @@ MLXQ_API int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32
                    uint64_t stream);
 
 /*
+ * Self-tests of the failure paths (no page entry; used by the tests).
+ *
+ * mlxq_selftest_wait_timeout: launches one warp on `stream` that waits,
+ * through the same bounded mbarrier wait every kernel uses, on a barrier that
+ * nothing completes.  After limit_us microseconds (1 .. 1,000,000) the wait
+ * gives up, sets the device status word and the kernel returns: nothing
+ * faults, traps or hangs, and the context stays usable.  The next
+ * mlxq_device_status then returns MLXQ_ERR_DEVICE_TIMEOUT (and clears it).
+ *
+ * mlxq_selftest_fail_alloc: makes the nth device allocation made by mlxq_load
+ * from now on fail as if cudaMalloc had run out of memory (nth = 1: the next
+ * one; 0 cancels).  mlxq_load then returns MLXQ_ERR_CUDA, frees what it had
+ * allocated and leaves the handle untouched.
+ */
+MLXQ_API int mlxq_selftest_wait_timeout(uint32_t limit_us, uint64_t stream);
+MLXQ_API int mlxq_selftest_fail_alloc(uint32_t nth);
+
+/*
  * mlxq_release (page: MlxInt8Weight::release).  Frees the three buffers of a
  * handle filled by mlxq_load and zeroes the handle.  The buffers are freed
  * exactly once: a second call on the same handle returns MLXQ_ERR_INVALID_ARG.

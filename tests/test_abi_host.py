@@ -252,3 +252,22 @@ def test_product_path_has_no_oracle_dependency():
                 text = open(os.path.join(dirpath, f)).read()
                 for needle in ("import oracle", "from oracle", "libmlxq_oracle", "mlxq_oracle"):
                     assert needle not in text, f"{f} references the oracle ({needle})"
+
+
+def test_load_injected_alloc_failure_leaves_handle_untouched():
+    # the first device allocation of the next load fails (no CUDA call is made)
+    mq.mlxq_selftest_fail_alloc(1)
+    try:
+        rc, w = _load_rc(_blob())
+    finally:
+        mq.mlxq_selftest_fail_alloc(0)
+    assert rc == mq.MLXQ_ERR_CUDA
+    assert "uploading" in mq.mlxq_last_error()
+    assert not w.packed and not w.scales and not w.biases and w.out_features == 0
+
+
+def test_selftest_wait_timeout_rejects_bad_limits():
+    for bad in (0, 1000001):
+        with pytest.raises(mq.MlxqError) as e:
+            mq.mlxq_selftest_wait_timeout(bad, 0)
+        assert e.value.code == mq.MLXQ_ERR_INVALID_ARG

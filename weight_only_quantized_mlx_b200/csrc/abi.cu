@@ -376,6 +376,17 @@ int launch_status(cudaError_t e, const char* what) {
 
 cudaStream_t as_stream(uint64_t s) { return reinterpret_cast<cudaStream_t>(static_cast<uintptr_t>(s)); }
 
+// mlxq_selftest_fail_alloc: the n-th device allocation of mlxq_load from now
+// fails as if cudaMalloc had run out (0: none).
+std::atomic<int> g_fail_alloc_in{0};
+bool take_injected_alloc_failure() {
+    int n = g_fail_alloc_in.load();
+    while (n > 0) {
+        if (g_fail_alloc_in.compare_exchange_weak(n, n - 1)) return n == 1;
+    }
+    return false;
+}
+
 }  // namespace
 
 const DeviceInfo& device_info() {
@@ -411,6 +422,18 @@ using namespace mlxq;
 extern "C" {
 
 const char* mlxq_last_error(void) { return g_err.c_str(); }
+
+int mlxq_selftest_fail_alloc(uint32_t nth) {
+    g_fail_alloc_in.store(static_cast<int>(nth > 1000000u ? 1000000u : nth));
+    return ok();
+}
+
+int mlxq_selftest_wait_timeout(uint32_t limit_us, uint64_t stream) {
+    if (limit_us < 1 || limit_us > 1000000u)
+        return fail(MLXQ_ERR_INVALID_ARG, "limit_us must be in [1, 1000000], got %u", limit_us);
+    return launch_status(launch_wait_timeout_selftest(1000ull * limit_us, as_stream(stream)),
+                         "wait-timeout self-test launch");
+}
 
 int mlxq_load(const void* blob, size_t blob_len, const char* base, uint32_t group_size, mlxq_weight* out) {
     if (!out) return fail(MLXQ_ERR_INVALID_ARG, "null output handle");
@@ -448,7 +471,8 @@ int mlxq_load(const void* blob, size_t blob_len, const char* base, uint32_t grou
     const TensorInfo* src[3] = {&tw, &tsc, &tb};
     void* ptr[3] = {nullptr, nullptr, nullptr};
     for (int i = 0; i < 3; ++i) {
-        cudaError_t e = cudaMalloc(&ptr[i], bytes[i] < 256 ? 256 : bytes[i]);
+        cudaError_t e = take_injected_alloc_failure() ? cudaErrorMemoryAllocation
+                                                      : cudaMalloc(&ptr[i], bytes[i] < 256 ? 256 : bytes[i]);
         if (e == cudaSuccess && bytes[i]) e = cudaMemcpy(ptr[i], data + src[i]->begin, bytes[i], cudaMemcpyHostToDevice);
         if (e != cudaSuccess) {
             for (int j = 0; j <= i; ++j)

@@ -65,13 +65,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns
-// false (and records a timeout) if it did not complete within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int* status) {
+// false (and records a timeout) if it did not complete within limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int* status,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+        if ((it & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) {
             atomicOr(status, MLXQ_STATUS_TIMEOUT);
             return false;
         }

@@ -93,6 +93,9 @@ cudaError_t launch_gemm_smallm(const WeightView& w, const void* X, void* Y, int6
 
 // tcgen05 tensor-core gemm.
 bool gemm_tc_supported(const WeightView& w, int64_t m, const void* X, const void* Y);
+// Self-test: one bounded wait that runs out after limit_ns (status word set).
+cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream);
+
 // Where the K-split partials of the tcgen05 gemm live: the library's
 // stream-ordered pool, or the static buffer of mlxq_gemm_noalloc.
 enum TcScratch { TC_SCRATCH_POOL = 0, TC_SCRATCH_STATIC = 1 };
