@@ -58,7 +58,7 @@ constexpr int kSSB = 2;                  // scale/bias slots
 struct TcParams {
     uint16_t* Y;
     int N, K, G, gs, m;
-    int BN, S, num_kb;
+    int BN, S, SX, num_kb;  // S: A-tile stages, SX: activation-tile stages
     int sg;          // k-blocks covered by one scale/bias box (8 * gs / 64)
     int sb_tma;      // 1: scales/biases by TMA boxes; 0 (rows not 16-byte multiples): direct loads
     int ks;          // K splits per tile (1: no split)
@@ -66,7 +66,7 @@ struct TcParams {
     unsigned int* counters;  // ks > 1: per-tile arrival counts, zero between launches
     const uint16_t* scales;
     const uint16_t* biases;
-    uint32_t stage_bytes, idesc, tmem_cols;
+    uint32_t idesc, tmem_cols;
     unsigned int* status;
 };
 
@@ -206,14 +206,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int num_units = num_tiles * p.ks;
     const int my_units = blockIdx.x < num_units ? (num_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-    // shared memory: S (A, X) stages | kSP packed slots | kSSB (scales, biases) slots | barriers
+    // shared memory: S A tiles | SX activation tiles | kSP packed slots |
+    // kSSB (scales, biases) slots | barriers.  The activation ring is the
+    // deeper one: its tiles come from L2/HBM, the A tiles from the dequant warps.
+    const int SX = p.SX;
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t p_base = sbase + static_cast<uint32_t>(S) * p.stage_bytes;
+    const uint32_t x_base = sbase + static_cast<uint32_t>(S) * kStageA;
+    const uint32_t p_base = x_base + static_cast<uint32_t>(SX) * stage_x;
     const uint32_t sb_base = p_base + kSP * kStageP;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * p.stage_bytes + kSP * kStageP +
-                                                 kSSB * 2 * kStageSB);
-    uint64_t* empty = full + S;
-    uint64_t* pfull = empty + S;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (sb_base + kSSB * 2 * kStageSB - sbase));
+    uint64_t* empty = full + S;      // A tile s: written (dequant) / read (MMA)
+    uint64_t* xfull = empty + S;     // activation tile: landed (TMA) / read (MMA)
+    uint64_t* xempty = xfull + SX;
+    uint64_t* pfull = xempty + SX;
     uint64_t* pempty = pfull + kSP;
     uint64_t* sbfull = pempty + kSP;
     uint64_t* sbempty = sbfull + kSSB;
@@ -221,8 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* acc_empty = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
     uint32_t* last_flag = tmem_slot + 1;  // epilogue: this CTA completed the tile
-    auto A_of = [&](int s) { return sbase + static_cast<uint32_t>(s) * p.stage_bytes; };
-    auto X_of = [&](int s) { return A_of(s) + kStageA; };
+    auto A_of = [&](int s) { return sbase + static_cast<uint32_t>(s) * kStageA; };
+    auto X_of = [&](int s) { return x_base + static_cast<uint32_t>(s) * stage_x; };
     auto P_of = [&](int s) { return p_base + static_cast<uint32_t>(s) * kStageP; };
     auto SC_of = [&](int s) { return sb_base + static_cast<uint32_t>(s) * 2u * kStageSB; };
     auto BI_of = [&](int s) { return SC_of(s) + kStageSB; };
@@ -241,8 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), 1 + kDequantWarps);
+            mbar_init(smem_u32(&full[s]), kDequantWarps);
             mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(smem_u32(&xfull[s]), 1);
+            mbar_init(smem_u32(&xempty[s]), 1);
         }
         for (int s = 0; s < kSP; ++s) {
             mbar_init(smem_u32(&pfull[s]), 1);
@@ -277,12 +286,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int tile, split, n0, m0, kb0, kb1;
                 unit_of(t, tile, split, n0, m0, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int s = it % S;
-                    if (it >= S && ok) ok = mbar_wait(smem_u32(&empty[s]), ((it / S) - 1) & 1, p.status);
-                    mbar_arrive_expect_tx(smem_u32(&full[s]), stage_x);
+                    const int s = it % SX;
+                    if (it >= SX && ok) ok = mbar_wait(smem_u32(&xempty[s]), ((it / SX) - 1) & 1, p.status);
+                    mbar_arrive_expect_tx(smem_u32(&xfull[s]), stage_x);
                     for (int r = 0; r < p.BN; r += kXBoxRows)
                         tma_load_2d(X_of(s) + static_cast<uint32_t>(r) * 128u, &tm_x, kb * kBK, m0 + r,
-                                    smem_u32(&full[s]), pol);
+                                    smem_u32(&xfull[s]), pol);
                 }
             }
         }
@@ -328,12 +337,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d0 = tmem_base, d1 = tmem_base + p.tmem_cols;
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
-                    const int s = it % S;
+                    const int s = it % S, sx = it % SX;
                     if (ok) ok = mbar_wait(smem_u32(&full[s]), (it / S) & 1, p.status);
+                    if (ok) ok = mbar_wait(smem_u32(&xfull[sx]), (it / SX) & 1, p.status);
                     tc_fence_after();
                     const uint64_t a0 = sw128_kmajor_desc(A_of(s));
                     const uint64_t a1 = sw128_kmajor_desc(A_of(s) + kHM * 128u);
-                    const uint64_t bd = sw128_kmajor_desc(X_of(s));
+                    const uint64_t bd = sw128_kmajor_desc(X_of(sx));
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         // advance 16 BF16 (32 bytes) along K inside the swizzled rows
@@ -342,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         umma_bf16(d1, a1 + 2u * kk, bd + 2u * kk, p.idesc, acc);
                     }
                     umma_commit(smem_u32(&empty[s]));
+                    umma_commit(smem_u32(&xempty[sx]));
                 }
                 umma_commit(smem_u32(acc_full));
             }
@@ -606,12 +617,16 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
     p.ks = pick_ks(tiles, p.num_kb, dev.sm_count);
     p.scales = w.scales;
     p.biases = w.biases;
-    p.stage_bytes = kStageA + static_cast<uint32_t>(p.BN) * 128u;
+    // two A tiles (filled on the SM by the dequant warps), then as many
+    // activation tiles (fetched from L2/HBM, ~2 us away) as shared memory holds
+    const size_t stage_x = static_cast<size_t>(p.BN) * 128u;
     const size_t fixed = 1024 /*alignment slack*/ + kSP * kStageP + kSSB * 2 * kStageSB + 64 * sizeof(uint64_t);
-    int S = static_cast<int>((static_cast<size_t>(dev.max_smem_optin) - fixed) / p.stage_bytes);
-    if (S > 6) S = 6;
-    if (S < 2) return cudaErrorInvalidValue;
-    p.S = S;
+    const size_t budget = static_cast<size_t>(dev.max_smem_optin);
+    p.S = 2;
+    if (fixed + 2 * kStageA + 2 * stage_x > budget) return cudaErrorInvalidValue;
+    int SX = static_cast<int>((budget - fixed - 2 * kStageA) / stage_x);
+    if (SX > 8) SX = 8;
+    p.SX = SX;
     p.idesc = (1u << 4)                                   // D: fp32
               | (1u << 7)                                 // A: BF16
               | (1u << 10)                                // B: BF16
@@ -631,7 +646,7 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
 
-    const size_t smem = static_cast<size_t>(S) * p.stage_bytes + fixed;
+    const size_t smem = 2 * kStageA + static_cast<size_t>(SX) * stage_x + fixed;
     static std::atomic<int> configured[64];
     cudaError_t e = ensure_dynamic_smem(k_gemm_tc, smem, configured);
     if (e != cudaSuccess) return e;
