@@ -236,17 +236,22 @@ def run_gpu(args):
     with ClockSampler(dev.index or 0) as clk:
         ms = time_region(graph.replay, args.steps, args.warmup, stream, world)
         ms_eager = time_region(lambda: step_on(s_ptr), args.steps, args.warmup, stream, world)
-        # e2e: the public call with host buffers; per step and pair, H2D of x
-        # from pinned memory, the gemv, D2H of y, all inside the timed region
-        xh = [x.cpu().pin_memory() for x in xs]
-        yh = [torch.empty(D_N, dtype=torch.bfloat16).pin_memory() for _ in range(N_PAIRS)]
-        xd = [torch.empty_like(x) for x in xs]
+        # e2e: the public call with host buffers.  Every step copies its 100
+        # activation vectors from pinned host memory in one H2D, makes the 100
+        # mlxq_gemv calls, and reads the 100 results back in one D2H, all
+        # inside the timed region (the copies are batched per step, as a
+        # caller holding a step's inputs would do).
+        xh = torch.stack([x.cpu() for x in xs]).pin_memory()          # [pairs, K]
+        yh = torch.empty(N_PAIRS, D_N, dtype=torch.bfloat16).pin_memory()
+        xd = torch.empty(N_PAIRS, D_K, dtype=torch.bfloat16, device=dev)
+        yd = torch.empty(N_PAIRS, D_N, dtype=torch.bfloat16, device=dev)
 
         def step_e2e():
-            for i in range(N_PAIRS):
-                xd[i].copy_(xh[i], non_blocking=True)
-                mq.mlxq_gemv(weights[i].handle, xd[i], ys[i], stream)
-                yh[i].copy_(ys[i], non_blocking=True)
+            with torch.cuda.stream(stream):
+                xd.copy_(xh, non_blocking=True)
+                for i in range(N_PAIRS):
+                    mq.mlxq_gemv(weights[i].handle, xd[i], yd[i], stream)
+                yh.copy_(yd, non_blocking=True)
 
         e2e_steps = max(1, args.steps // 4)
         ms_e2e = time_region(step_e2e, e2e_steps, max(3, args.warmup), stream, world)

@@ -52,6 +52,9 @@ struct MmaParams {
     uint32_t box_bytes;     // R16 * 128
     uint32_t sb_bytes;      // R16 * gpk * 2, rounded up to 128
     uint32_t stage_bytes;
+    uint32_t x_off;         // m > 1: offset of the stage's activation boxes (1024-aligned)
+    uint32_t xbox_bytes;    // m > 1: one [8 NT rows x 64 columns] BF16 box, 128-byte swizzle
+    uint32_t x_tx;          // m > 1: activation bytes per stage (0 for m == 1)
     uint32_t xs_bytes;      // activation staging (m == 1)
     unsigned int* status;
 };
@@ -86,10 +89,13 @@ __device__ __forceinline__ float silu_f32(float t) { return t / (1.0f + expf(-t)
 // NB: 128-code boxes per stage; consumer warp w takes box w % NB and row
 // pairs p = w / NB + j * (kWarps / NB).  PW: most pairs one warp holds.
 // NT: activation column tiles of 8 (m <= 8 * NT).
-template <int MODE, int NB, int PW, int NT>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_stream_mma(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_scales,
-                 const __grid_constant__ CUtensorMap tm_biases, const MmaParams p) {
+//
+// XS: m > 1, the activations arrive by TMA with each stage (tm_x); without
+// it (m == 1) they are staged once per CTA from global memory.
+template <int MODE, int NB, int PW, int NT, bool XS>
+__device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const CUtensorMap& tm_scales,
+                                           const CUtensorMap& tm_biases, const CUtensorMap* tm_x,
+                                           const MmaParams& p) {
     constexpr int kKB = 128 * NB;
     constexpr int kSub = kWarps / NB;  // row-pair subsets
     extern __shared__ uint8_t smem_raw[];
@@ -133,8 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_prefetch_l2_2d(&tm_scales, kb * p.gpk, r0);
                 tma_prefetch_l2_2d(&tm_biases, kb * p.gpk, r0);
             }
+            if constexpr (XS) prefetch_tmap(tm_x);
             pdl_wait();
             const uint64_t pol = policy_evict_first();
+            [[maybe_unused]] const uint64_t pol_x = XS ? policy_evict_last() : 0ull;  // every CTA reads the same activations
             bool ok = true;
             for (int kb = 0; kb < p.num_kb; ++kb) {
                 const int s = kb % S;
@@ -145,11 +153,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t bar = smem_u32(&full[s]);
                 const uint32_t st = stage_of(s);
                 mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * 128u * p.R +
-                                               2u * static_cast<uint32_t>(p.R) * p.gpk * 2u);
+                                               2u * static_cast<uint32_t>(p.R) * p.gpk * 2u + p.x_tx);
                 for (int b = 0; b < nbox; ++b)
                     tma_load_2d(st + static_cast<uint32_t>(b) * p.box_bytes, &tm_packed, col0 + 128 * b, r0, bar, pol);
                 tma_load_2d(st + NB * p.box_bytes, &tm_scales, kb * p.gpk, r0, bar, pol);
                 tma_load_2d(st + NB * p.box_bytes + p.sb_bytes, &tm_biases, kb * p.gpk, r0, bar, pol);
+                if constexpr (XS)  // the stage's activation columns, all 8 NT rows (zero past m and K)
+                    for (int j = 0; j < kKB / 64; ++j)
+                        tma_load_2d(st + p.x_off + static_cast<uint32_t>(j) * p.xbox_bytes, tm_x, col0 + 64 * j, 0, bar,
+                                    pol_x);
             }
         }
         return;
@@ -255,24 +267,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int kcs = kin ? kc : 0;  // a valid address when out of range
             // B fragments: activation column (8 t + g) at this lane's 16 codes
             uint32_t b[NT][8];
+            if constexpr (!XS) {
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                uint4 v0, v1;
-                if (p.m == 1) {
-                    const uint32_t base = xs + xrow_off + 2u * static_cast<uint32_t>(kcs);
-                    v0 = lds128(base);
-                    v1 = lds128(base + 16);
-                } else {
-                    const int colr = colv[t] ? 8 * t + g : 0;
-                    const uint16_t* xr = p.X + static_cast<int64_t>(colr) * p.K + kcs;
-                    v0 = ldg_nc_v4(xr);
-                    v1 = ldg_nc_v4(xr + 8);
+                for (int t = 0; t < NT; ++t) {
+                    uint4 v0, v1;
+                    if (p.m == 1) {
+                        const uint32_t base = xs + xrow_off + 2u * static_cast<uint32_t>(kcs);
+                        v0 = lds128(base);
+                        v1 = lds128(base + 16);
+                    } else {
+                        const int colr = colv[t] ? 8 * t + g : 0;
+                        const uint16_t* xr = p.X + static_cast<int64_t>(colr) * p.K + kcs;
+                        v0 = ldg_nc_v4(xr);
+                        v1 = ldg_nc_v4(xr + 8);
+                    }
+                    const bool live = kin && colv[t];
+                    b[t][0] = live ? v0.x : 0u; b[t][1] = live ? v0.y : 0u;
+                    b[t][2] = live ? v0.z : 0u; b[t][3] = live ? v0.w : 0u;
+                    b[t][4] = live ? v1.x : 0u; b[t][5] = live ? v1.y : 0u;
+                    b[t][6] = live ? v1.z : 0u; b[t][7] = live ? v1.w : 0u;
                 }
-                const bool live = kin && colv[t];
-                b[t][0] = live ? v0.x : 0u; b[t][1] = live ? v0.y : 0u;
-                b[t][2] = live ? v0.z : 0u; b[t][3] = live ? v0.w : 0u;
-                b[t][4] = live ? v1.x : 0u; b[t][5] = live ? v1.y : 0u;
-                b[t][6] = live ? v1.z : 0u; b[t][7] = live ? v1.w : 0u;
+            } else {
+                // staged by TMA with the stage (zero past m and K): 64-column
+                // box 2 box + ci, row 8 t + g, 16-byte chunks 2 tq and 2 tq + 1
+                // placed by the 128-byte swizzle (chunk ^ row % 8; row % 8 == g)
+                const uint32_t xb = st + p.x_off + static_cast<uint32_t>(2 * box + ci) * p.xbox_bytes;
+                const uint32_t c0 = static_cast<uint32_t>((2 * tq) ^ g) << 4;
+                const uint32_t c1 = static_cast<uint32_t>((2 * tq + 1) ^ g) << 4;
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    const uint32_t ra = xb + static_cast<uint32_t>(8 * t + g) * 128u;
+                    const uint4 v0 = lds128(ra + c0), v1 = lds128(ra + c1);
+                    b[t][0] = v0.x; b[t][1] = v0.y; b[t][2] = v0.z; b[t][3] = v0.w;
+                    b[t][4] = v1.x; b[t][5] = v1.y; b[t][6] = v1.z; b[t][7] = v1.w;
+                }
             }
             const uint32_t sgo = ci ? sgrp1 : 0u;
             // row pairs in groups of two: load both, then interleave the MMAs
@@ -372,32 +400,57 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int MODE, int NB, int PW, int NT>
-cudaError_t launch_t(const TensorMaps3& tm, const MmaParams& p, int grid, size_t smem, cudaStream_t stream) {
-    auto kern = k_stream_mma<MODE, NB, PW, NT>;
-    static std::atomic<int> configured[64];
-    cudaError_t e = ensure_dynamic_smem(kern, smem, configured);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, tm.packed, tm.scales, tm.biases, p);
+__global__ void __launch_bounds__(kThreads, 1)
+    k_stream_mma(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_scales,
+                 const __grid_constant__ CUtensorMap tm_biases, const MmaParams p) {
+    stream_mma<MODE, NB, PW, NT, false>(tm_packed, tm_scales, tm_biases, nullptr, p);
+}
+
+template <int NB, int PW, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_stream_mma_xs(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_scales,
+                    const __grid_constant__ CUtensorMap tm_biases, const __grid_constant__ CUtensorMap tm_x,
+                    const MmaParams p) {
+    stream_mma<GEMV_PLAIN, NB, PW, NT, true>(tm_packed, tm_scales, tm_biases, &tm_x, p);
+}
+
+template <int MODE, int NB, int PW, int NT>
+cudaError_t launch_t(const TensorMaps3& tm, const CUtensorMap& tmx, const MmaParams& p, int grid, size_t smem,
+                     cudaStream_t stream) {
+    cudaError_t e;
+    if (p.x_tx) {  // m > 1
+        auto kern = k_stream_mma_xs<NB, PW, NT>;
+        static std::atomic<int> configured[64];
+        e = ensure_dynamic_smem(kern, smem, configured);
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, tm.packed, tm.scales, tm.biases, tmx, p);
+    } else {
+        auto kern = k_stream_mma<MODE, NB, PW, NT>;
+        static std::atomic<int> configured[64];
+        e = ensure_dynamic_smem(kern, smem, configured);
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, tm.packed, tm.scales, tm.biases, p);
+    }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 template <int MODE, int NT>
-cudaError_t launch_pw(const TensorMaps3& tm, const MmaParams& p, int nb, int npair, int grid, size_t smem,
-                      cudaStream_t stream) {
+cudaError_t launch_pw(const TensorMaps3& tm, const CUtensorMap& tmx, const MmaParams& p, int nb, int npair, int grid,
+                      size_t smem, cudaStream_t stream) {
     // rows per CTA are capped by NT on the host, so at most 4 / NT pairs per warp
     const int sub = kWarps / nb;
     const int pw = (npair + sub - 1) / sub;
     if (nb == 8) {
-        if (pw <= 1) return launch_t<MODE, 8, 1, NT>(tm, p, grid, smem, stream);
+        if (pw <= 1) return launch_t<MODE, 8, 1, NT>(tm, tmx, p, grid, smem, stream);
         if constexpr (NT <= 2) {
-            if (pw <= 2) return launch_t<MODE, 8, 2, NT>(tm, p, grid, smem, stream);
+            if (pw <= 2) return launch_t<MODE, 8, 2, NT>(tm, tmx, p, grid, smem, stream);
         }
-        if constexpr (NT == 1) return launch_t<MODE, 8, 4, NT>(tm, p, grid, smem, stream);
+        if constexpr (NT == 1) return launch_t<MODE, 8, 4, NT>(tm, tmx, p, grid, smem, stream);
         return cudaErrorInvalidValue;
     }
-    if (pw <= 1) return launch_t<MODE, 4, 1, NT>(tm, p, grid, smem, stream);
-    if constexpr (NT <= 2) return launch_t<MODE, 4, 2, NT>(tm, p, grid, smem, stream);
+    if (pw <= 1) return launch_t<MODE, 4, 1, NT>(tm, tmx, p, grid, smem, stream);
+    if constexpr (NT <= 2) return launch_t<MODE, 4, 2, NT>(tm, tmx, p, grid, smem, stream);
     return cudaErrorInvalidValue;
 }
 
@@ -453,6 +506,12 @@ cudaError_t launch_stream_mma(const WeightView& w, int mode, int64_t m, const vo
     p.sb_bytes = (static_cast<uint32_t>(p.R16) * p.gpk * 2u + 127u) / 128u * 128u;
     p.stage_bytes = static_cast<uint32_t>(nb) * p.box_bytes + 2u * p.sb_bytes;
     p.stage_bytes = (p.stage_bytes + 1023u) / 1024u * 1024u;  // keep every box 1024-byte aligned
+    if (m > 1) {  // the stage's activation slice: kKB / 64 boxes of [8 nt rows x 64 columns]
+        p.x_off = p.stage_bytes;
+        p.xbox_bytes = static_cast<uint32_t>(8 * nt) * 128u;
+        p.x_tx = static_cast<uint32_t>(kKB / 64) * p.xbox_bytes;
+        p.stage_bytes += p.x_tx;
+    }
     p.xs_bytes = (m == 1) ? static_cast<uint32_t>((mode == GEMV_PLAIN ? 2 : 4) * w.K + 127) / 128u * 128u : 0u;
     const uint32_t red_bytes = kWarps * static_cast<uint32_t>(m) * static_cast<uint32_t>(p.R16) * 4u;
     const size_t fixed = 1024 + p.xs_bytes + 2 * 16 * sizeof(uint64_t);
@@ -474,14 +533,19 @@ cudaError_t launch_stream_mma(const WeightView& w, int mode, int64_t m, const vo
 
     TensorMaps3 maps;
     if (!weight_tensor_maps(w, p.R, 128, CU_TENSOR_MAP_SWIZZLE_128B, p.gpk, &maps)) return cudaErrorInvalidValue;
+    CUtensorMap tmx = maps.packed;  // m == 1: not read
+    if (m > 1 && !encode_2d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(w.K),
+                            static_cast<uint64_t>(m), static_cast<uint64_t>(w.K) * 2, 64,
+                            static_cast<uint32_t>(8 * nt), CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
     const int grid = static_cast<int>((w.N + p.R - 1) / p.R);
     const int npair = p.R16 / 16;
-    if (nt == 2) return launch_pw<GEMV_PLAIN, 2>(maps, p, nb, npair, grid, smem, stream);
-    if (nt == 4) return launch_pw<GEMV_PLAIN, 4>(maps, p, nb, npair, grid, smem, stream);
+    if (nt == 2) return launch_pw<GEMV_PLAIN, 2>(maps, tmx, p, nb, npair, grid, smem, stream);
+    if (nt == 4) return launch_pw<GEMV_PLAIN, 4>(maps, tmx, p, nb, npair, grid, smem, stream);
     switch (mode) {
-        case GEMV_PLAIN: return launch_pw<GEMV_PLAIN, 1>(maps, p, nb, npair, grid, smem, stream);
-        case GEMV_SILU: return launch_pw<GEMV_SILU, 1>(maps, p, nb, npair, grid, smem, stream);
-        default: return launch_pw<GEMV_SILU_RESID, 1>(maps, p, nb, npair, grid, smem, stream);
+        case GEMV_PLAIN: return launch_pw<GEMV_PLAIN, 1>(maps, tmx, p, nb, npair, grid, smem, stream);
+        case GEMV_SILU: return launch_pw<GEMV_SILU, 1>(maps, tmx, p, nb, npair, grid, smem, stream);
+        default: return launch_pw<GEMV_SILU_RESID, 1>(maps, tmx, p, nb, npair, grid, smem, stream);
     }
 }
 
