@@ -1,5 +1,5 @@
-// Stream kernel for the m <= 8 rows of the "MlxInt8Weight" page's gemv,
-// gemv_silu_gate, gemv_silu_gate_resid and small-m gemm, with the
+// Stream kernels for the "MlxInt8Weight" page's gemv, gemv_silu_gate,
+// gemv_silu_gate_resid (m = 1) and small-m gemm (m <= 32), with the
 // multiply-adds on the tensor pipe.
 //
 // Why: the work is HBM-bound, one weight byte per code, and at ~6.5 TB/s a
@@ -9,25 +9,28 @@
 // dequantisation (byte -> fp32 via the 2^23 exponent trick, fp32 fma with
 // scale and bias, RNE to BF16 - the exact BF16 weight of dequantize_to); the
 // products and fp32 sums run in mma.sync m16n8k16 (BF16 in, fp32
-// accumulate), with the dequantised weights feeding the B fragment straight
-// from registers.
+// accumulate), with the dequantised weights going straight from registers
+// into the A fragment.
 //
-// Layout (per MMA): A = activations, 16 x 16 (row i = activation row i,
-// zero-padded), B = 16 codes x 8 weight rows, D = 16 x 8.  Lane (g, t) owns
-// weight row g of the octet and a 16-code chunk; its four words feed four
-// MMAs, the k order inside each MMA being a fixed permutation that A and B
-// share (sums are order-free up to fp32 rounding).
+// Layout (per MMA): A = dequantised weights, 16 rows x 16 codes (lane (g, t)
+// holds rows g and g + 8 of a row pair); B = activations, 16 codes x 8
+// activation rows; D = 16 weight rows x 8 activation rows.  The k order
+// inside each MMA is a fixed permutation that A and B share (sums are
+// order-free up to fp32 rounding).
 //
 // Data movement: one CTA owns R consecutive weight rows (R ~ N / #SMs, so HBM
-// work is balanced to one row); a producer lane streams K in blocks of
-// 128 * W codes with 2-D tensor copies: W boxes of [R rows x 128 bytes] with
-// the 128-byte swizzle (conflict-free fragment loads), plus the matching
-// [R x groups] scale and bias boxes.  Consumer warp w owns box w of every
-// stage.  For gemv, x (or, for the silu variants, h = silu(gate)*up split
-// into a BF16 high part and a BF16 low part, so h keeps ~16 bits and is never
-// written to global memory) sits in shared memory; for m > 1 the activation
-// fragments are read from global memory (L2-resident).  The warps' partial
-// results are summed in shared memory in a fixed order.
+// work is balanced to one row); a producer lane streams K in stages of
+// 128 * NB codes with 2-D tensor copies: NB boxes of [R rows x 128 bytes]
+// with the 128-byte swizzle (conflict-free fragment loads), plus the
+// matching [R x groups] scale and bias boxes.  Consumer warp w takes box
+// w % NB of every stage for its subset of row pairs.  Activations:
+//   m == 1 (k_stream_mma): x - or, for the silu variants, h = silu(gate)*up
+//          split into a BF16 high and a BF16 low part, so h keeps ~16 bits
+//          and is never written to global memory - is staged once per CTA;
+//   m > 1 (k_stream_mma_xs): each stage's activation slice arrives by TMA
+//          with its weight boxes ([8 NT rows x 64 columns] boxes, 128-byte
+//          swizzle, zero past m and K).
+// The warps' partial results are summed in shared memory in a fixed order.
 #include "device_common.cuh"
 #include "kernels.h"
 #include "tensor_map.h"
