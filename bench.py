@@ -143,6 +143,13 @@ def dist_env():
     return rank, world, local
 
 
+def rank_pair_seeds(rank: int):
+    """Seeds of the decode pairs rank `rank` streams: ranks own disjoint,
+    consecutive blocks of N_PAIRS problems (weak scaling, no data-path
+    collective)."""
+    return [rank * N_PAIRS + i for i in range(N_PAIRS)]
+
+
 def max_over_ranks(value: float, world: int, device=None) -> float:
     if world == 1:
         return value
@@ -204,8 +211,8 @@ def run_gpu(args):
 
     # ---- headline: 100 decode gemvs, inputs resident in HBM -----------------
     weights, xs = [], []
-    for i in range(N_PAIRS):
-        p, s, b, x = synth.decode_pair(rank * N_PAIRS + i, D_N, D_K, D_GS)
+    for seed in rank_pair_seeds(rank):
+        p, s, b, x = synth.decode_pair(seed, D_N, D_K, D_GS)
         weights.append(upload_weight(mq, p, s, b, D_GS))
         xs.append(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev))
     ys = [torch.empty(D_N, dtype=torch.bfloat16, device=dev) for _ in range(N_PAIRS)]
