@@ -198,7 +198,9 @@ MLXQ_API const char* mlxq_last_error(void);
  * library's device status word.  Returns MLXQ_OK, or MLXQ_ERR_DEVICE_TIMEOUT
  * if some kernel since the last check gave up a bounded wait (its outputs are
  * then not valid), or MLXQ_ERR_CUDA.  Kernels never hang or trap on a stalled
- * pipeline: they record the timeout here and return.
+ * pipeline: they record the timeout here and return.  On a timeout it also
+ * zeroes the tile counters of mlxq_gemm_noalloc's static scratch, which an
+ * interrupted K split may have left raised.
  */
 MLXQ_API int mlxq_device_status(void);
 

@@ -630,7 +630,14 @@ int mlxq_device_status(void) {
     e = cudaMemcpyFromSymbol(&v, g_status_word, sizeof(v));
     if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
     if (e != cudaSuccess) return launch_status(e, "reading the device status word");
-    if (v) return fail(MLXQ_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded pipeline wait (status 0x%x)", v);
+    if (v) {
+        // a split gemm may have stopped between raising and clearing its tile
+        // counters: zero the static scratch's counters so mlxq_gemm_noalloc
+        // starts clean again
+        e = reset_static_scratch_counters();
+        if (e != cudaSuccess) return launch_status(e, "resetting the static scratch counters");
+        return fail(MLXQ_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded pipeline wait (status 0x%x)", v);
+    }
     return ok();
 }
 

@@ -563,6 +563,19 @@ cudaError_t static_scratch_base(int device, unsigned char** out) {
     return cudaSuccess;
 }
 
+// Synchronous: called from mlxq_device_status after a device-wide sync.
+}  // namespace
+
+cudaError_t reset_static_scratch_counters() {
+    const DeviceInfo& dev = device_info();
+    unsigned char* base = nullptr;
+    cudaError_t e = static_scratch_base(dev.device, &base);
+    if (e != cudaSuccess) return e;
+    return cudaMemset(base, 0, kCounterBytes);
+}
+
+namespace {
+
 // K splits per tile: only when the tiles alone leave SMs idle; as many as
 // keep every split in one wave (units <= SMs) and >= kMinKbPerSplit long.
 int pick_ks(int64_t tiles, int num_kb, int sm_count) {

@@ -100,6 +100,8 @@ cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream
 // stream-ordered pool, or the static buffer of mlxq_gemm_noalloc.
 enum TcScratch { TC_SCRATCH_POOL = 0, TC_SCRATCH_STATIC = 1 };
 constexpr size_t kStaticScratchBytes = MLXQ_STATIC_SCRATCH_BYTES;
+// Zero the tile counters of the static scratch (after a timed-out wait).
+cudaError_t reset_static_scratch_counters();
 // Scratch bytes a tcgen05 gemm of this shape needs (0: no K split).
 size_t gemm_tc_scratch_bytes(const WeightView& w, int64_t m);
 cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream,
