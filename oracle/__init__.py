@@ -48,6 +48,7 @@ def _signatures():
         "oracle_silu_mul": (None, [u16p, u16p, i64, u16p]),
         "oracle_gemm_f64": (None, W + [u16p, i64, f64p]),
         "oracle_gemm": (None, W + [u16p, i64, u16p]),
+        "oracle_quantize": (None, [u16p, i64, i64, i64, u32p, u16p, u16p]),
     }
 
 
@@ -136,6 +137,20 @@ class Oracle:
         w = np.empty((N, K), np.float32)
         self.L.oracle_dequant_f32(*args, _p(w, ctypes.c_float))
         return w
+
+    def quantize(self, w_bits, gs):
+        """BF16 W [N, K] (bit patterns) -> (packed uint32 [N, K/4], scales,
+        biases uint16 [N, K/gs]) by per-group min/max affine codes."""
+        w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+        N, K = w.shape
+        if gs <= 0 or K % gs or K % 4 or gs % 4:
+            raise ValueError("quantize needs gs | K and 4 | gs")
+        packed = np.empty((N, K // 4), np.uint32)
+        scales = np.empty((N, K // gs), np.uint16)
+        biases = np.empty((N, K // gs), np.uint16)
+        self.L.oracle_quantize(_p(w, ctypes.c_uint16), N, K, gs, _p(packed, ctypes.c_uint32),
+                               _p(scales, ctypes.c_uint16), _p(biases, ctypes.c_uint16))
+        return packed, scales, biases
 
     def dequant(self, packed, scales, biases, gs) -> np.ndarray:
         """BF16 bit patterns of the dequantised weight, [N, K] row-major."""

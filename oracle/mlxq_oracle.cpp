@@ -21,6 +21,11 @@
 //   * "gemv_silu_gate": y = W (silu(gate) * up).
 //   * "gemv_silu_gate_resid": y[n] = x_resid[n] + sum_k W[n,k]*(silu(gate[k])*up[k]).
 //   * "gemm": Y = X W^T, X [m, in_features], Y [m, out_features].
+//   * quantize (no page entry: the inverse of the format, which the head
+//     builder of the model pages applies to BF16 projections; the pages give
+//     no algorithm).  Parity unpinned against the pages: the min/max affine
+//     reading below is pinned by invariants only (grid identity, error bound,
+//     constant groups).
 //
 // Readings taken where the page is silent (each is listed in the design doc):
 //   * q[n,k] is byte (k mod 4) of word packed[n, k/4], little-endian
@@ -31,7 +36,13 @@
 //   * silu(t) = t / (1 + exp(-t)), in fp64; silu(gate)*up is NOT rounded.
 //   * Each output is rounded once, fp64 -> BF16, round to nearest even.
 //
-// Parity status of every function: pinned (see tests/test_oracle.py).
+// Parity status: every function pinned (see tests/test_oracle.py), except
+// that oracle_quantize's algorithm itself has no page to be checked against.
+//
+// quantize reading (per row, per group of gs columns, all fp32, each
+// operation rounded to nearest even, no fused operations):
+//   lo = min, hi = max of the group;  s = bf16((hi - lo) / 255);
+//   b = bf16(lo);  q = clamp(rint((w - b) / s), 0, 255), or q = 0 if s == 0.
 
 #include <cmath>
 #include <cstdint>
@@ -243,6 +254,45 @@ void oracle_gemm(const uint32_t* packed, const uint16_t* scales,
     std::vector<double> acc(static_cast<size_t>(m * N));
     oracle_gemm_f64(packed, scales, biases, N, K, gs, X, m, acc.data());
     for (int64_t t = 0; t < m * N; ++t) Y[t] = f64_to_bf16(acc[t]);
+}
+
+// quantize: BF16 W [N, K] -> packed codes, BF16 scales and biases [N, K/gs].
+void oracle_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t gs, uint32_t* packed,
+                     uint16_t* scales, uint16_t* biases) {
+    const int64_t G = K / gs;
+    std::vector<uint8_t> q(static_cast<size_t>(K));
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < G; ++g) {
+            const uint16_t* src = w + n * K + g * gs;
+            float lo = bf16_to_f32(src[0]), hi = lo;
+            for (int64_t j = 1; j < gs; ++j) {
+                const float v = bf16_to_f32(src[j]);
+                if (v < lo) lo = v;
+                if (v > hi) hi = v;
+            }
+            const float range = hi - lo;
+            const uint16_t sb = f32_to_bf16(range / 255.0f);
+            const uint16_t bb = f32_to_bf16(lo);
+            const float sf = bf16_to_f32(sb), bf = bf16_to_f32(bb);
+            for (int64_t j = 0; j < gs; ++j) {
+                float c = 0.0f;
+                if (sf != 0.0f) {
+                    const float d = bf16_to_f32(src[j]) - bf;
+                    c = std::nearbyint(d / sf);  // default rounding: to nearest, ties to even
+                    if (c < 0.0f) c = 0.0f;
+                    if (c > 255.0f) c = 255.0f;
+                }
+                q[static_cast<size_t>(g * gs + j)] = static_cast<uint8_t>(c);
+            }
+            scales[n * G + g] = sb;
+            biases[n * G + g] = bb;
+        }
+        for (int64_t k4 = 0; k4 < K / 4; ++k4) {
+            uint32_t word = 0;
+            for (int j = 0; j < 4; ++j) word |= static_cast<uint32_t>(q[static_cast<size_t>(4 * k4 + j)]) << (8 * j);
+            packed[n * (K / 4) + k4] = word;
+        }
+    }
 }
 
 }  // extern "C"

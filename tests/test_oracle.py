@@ -295,10 +295,65 @@ def pin_gemm_rows_are_gemv(o: Oracle):
         assert np.array_equal(Y[i], o.gemv(packed, scales, biases, gs, X[i]))
 
 
+# ---- quantize (the inverse of the format; the pages give no algorithm, so
+# these pins check invariants of the min/max affine reading) ----------------
+def pin_quantize_grid_identity(o: Oracle):
+    # Weights that already lie on a grid s = 2^-e, b = -128 s, with every group
+    # holding both code 0 and code 255: the group range is exactly 255 s, so
+    # quantize must give back s, b and every code exactly.
+    g = np.random.default_rng(40)
+    N, K, gs = 3, 96, 32
+    q = g.integers(0, 256, size=(N, K), dtype=np.uint8)
+    q[:, ::gs] = 0
+    q[:, 1::gs] = 255
+    for e in (2, 8, 14):
+        s = bf16_torch(np.full((N, K // gs), 2.0 ** -e))
+        b = bf16_torch(np.full((N, K // gs), -128 * 2.0 ** -e))
+        w = o.dequant(pack_le(q), s, b, gs)
+        p2, s2, b2 = o.quantize(w, gs)
+        assert np.array_equal(s2, s) and np.array_equal(b2, b), e
+        assert np.array_equal(p2, pack_le(q)), e
+
+
+def pin_quantize_error_bound(o: Oracle):
+    # Round trip of arbitrary BF16 weights: each code is the nearest grid
+    # point, so |W' - W| <= s / 2, except at the top of a group whose BF16
+    # scale was rounded down, where code 255 falls short of the group maximum
+    # by hi - (b + 255 s); plus the BF16 rounding of W' (half an ulp, <= 2^-8 |W'|) and of
+    # the stored bias.  The group minimum maps to code 0.
+    g = np.random.default_rng(41)
+    N, K, gs = 4, 256, 64
+    w = bf16_torch(g.standard_normal((N, K)) * 0.05)
+    p, s, b = o.quantize(w, gs)
+    w2 = bf16_bits_to_f64(o.dequant(p, s, b, gs))
+    wf = bf16_bits_to_f64(w)
+    sf = np.repeat(bf16_bits_to_f64(s), gs, axis=1)
+    bf = np.repeat(bf16_bits_to_f64(b), gs, axis=1)
+    lo = np.repeat(wf.reshape(N, K // gs, gs).min(axis=2), gs, axis=1)
+    hi = np.repeat(wf.reshape(N, K // gs, gs).max(axis=2), gs, axis=1)
+    top = np.maximum(sf / 2, hi - (bf + 255 * sf))
+    assert np.all(np.abs(w2 - wf) <= top + 2.0 ** -8 * np.abs(w2) + np.abs(bf - lo) + 1e-12)
+    codes = o.unpack(p).reshape(N, K // gs, gs)
+    assert np.all(codes[np.arange(N)[:, None], np.arange(K // gs)[None, :],
+                        wf.reshape(N, K // gs, gs).argmin(axis=2)] == 0)
+
+
+def pin_quantize_constant_group(o: Oracle):
+    # A constant group has range 0: scale 0, bias = the value, codes 0, and
+    # dequantisation returns the value exactly.
+    w = bf16_torch(np.array([[0.375] * 16 + [-2.5] * 16]))
+    p, s, b = o.quantize(w, 16)
+    assert np.array_equal(s, np.zeros((1, 2), np.uint16))
+    assert np.array_equal(bf16_bits_to_f64(b), np.array([[0.375, -2.5]]))
+    assert np.array_equal(p, np.zeros((1, 8), np.uint32))
+    assert np.array_equal(o.dequant(p, s, b, 16), w)
+
+
 PINS = [pin_bf16_f32_table, pin_bf16_f64_table, pin_bf16_two_routes_agree, pin_unpack_word,
         pin_identity_scale, pin_centred_scale, pin_group_index, pin_worked_example,
         pin_bruteforce, pin_integer_exact, pin_silu_closed_forms, pin_silu_gate_zero,
-        pin_silu_gate_structure, pin_gemm_rows_are_gemv]
+        pin_silu_gate_structure, pin_gemm_rows_are_gemv, pin_quantize_grid_identity,
+        pin_quantize_error_bound, pin_quantize_constant_group]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -321,6 +376,9 @@ MUTANTS = {
                         "if (std::isnan(v)) return 0x7FC0u;\n    return f32_to_bf16(static_cast<float>(v));"),
     "x_index_shift": ("acc += row[k] * static_cast<double>(bf16_to_f32(x[k]));",
                       "acc += row[k] * static_cast<double>(bf16_to_f32(x[(k + 1) % K]));"),
+    "quant_divisor_256": ("f32_to_bf16(range / 255.0f)", "f32_to_bf16(range / 256.0f)"),
+    "quant_bias_from_max": ("const uint16_t bb = f32_to_bf16(lo);", "const uint16_t bb = f32_to_bf16(hi);"),
+    "quant_round_down": ("c = std::nearbyint(d / sf);", "c = std::floor(d / sf);"),
 }
 
 
