@@ -340,6 +340,22 @@ def measure_rows(mq, torch, synth, dev, stream, dec_weights, peaks, args):
     rows["dequant_4096x4096"] = {"value": round(gbs, 1), "unit": "GB/s", "frac_hbm": round(gbs / hbm, 4),
                                  "bytes_per_launch": b // len(dec_weights)}
 
+    # quantize: BF16 [4096, 4096] -> codes + tables, 8 sources rotating (268 MB)
+    qsrc = [torch.randn(D_N, D_K, device=dev).to(torch.bfloat16) * 0.04 for _ in range(8)]
+    qdst = upload_weight(mq, *synth.weight(synth.rng(5000), D_N, D_K, D_GS), D_GS)
+    qturn = [0]
+
+    def quant():
+        mq.mlxq_quantize(qsrc[qturn[0] % len(qsrc)], qdst.handle, stream)
+        qturn[0] += 1
+    ms = time_region(quant, steps, warm, stream, 1)
+    b = 2 * D_N * D_K + D_N * D_K + 4 * D_N * D_K // D_GS
+    gbs = b / (ms * 1e-3) / 1e9
+    rows["quantize_4096x4096"] = {"value": round(gbs, 1), "unit": "GB/s", "frac_hbm": round(gbs / hbm, 4),
+                                  "bytes_per_launch": b}
+    qdst.release()
+    del qsrc
+
     # fused decode MLP: gate, up (14336x4096) then silu_gate_resid down (4096x14336)
     D, F, gs = 4096, 14336, 64
     mlps = []

@@ -166,6 +166,21 @@ MLXQ_API int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32
                    uint64_t stream);
 
 /*
+ * mlxq_quantize (no page entry: the inverse of the format; the pages give no
+ * quantizer algorithm, so the plain per-group min/max affine one is used).
+ * w_bf16: BF16 [out_features, in_features] row-major, device.  dst: a handle
+ * whose packed/scales/biases point at caller-owned device buffers of the
+ * format's sizes and whose dimensions and group_size (a multiple of 4, dividing
+ * in_features) describe w.  Per row and group, in fp32, each operation
+ * rounded to nearest even:
+ *   s = bf16((max - min) / 255), b = bf16(min),
+ *   q = clamp(rint((w - b) / s), 0, 255)  (all q = 0 when s == 0),
+ * codes little-endian in the words.  The result is a weight every other call
+ * takes.  Source and destination must not overlap (MLXQ_ERR_INVALID_ARG).
+ */
+MLXQ_API int mlxq_quantize(const void* w_bf16, const mlxq_weight* dst, uint64_t stream);
+
+/*
  * Self-tests of the failure paths (no page entry; used by the tests).
  *
  * mlxq_selftest_wait_timeout: launches one warp on `stream` that waits,

@@ -271,3 +271,23 @@ def test_selftest_wait_timeout_rejects_bad_limits():
         with pytest.raises(mq.MlxqError) as e:
             mq.mlxq_selftest_wait_timeout(bad, 0)
         assert e.value.code == mq.MLXQ_ERR_INVALID_ARG
+
+
+def test_quantize_validation_before_any_launch():
+    # host checks only: fake (non-null, aligned) device addresses, nothing launched
+    N, K = 8, 64
+    base = 1 << 40
+    def handle(gs, packed=base, scales=base + (1 << 20), biases=base + (2 << 20)):
+        return mq.mlxq_weight(packed, scales, biases, N, K, gs)
+    w = base + (3 << 20)
+    for gs, code in ((6, mq.MLXQ_ERR_GROUP_SIZE), (2, mq.MLXQ_ERR_UNSUPPORTED), (0, mq.MLXQ_ERR_GROUP_SIZE)):
+        with pytest.raises(mq.MlxqError) as e:
+            mq.mlxq_quantize(w, handle(gs), 0)
+        assert e.value.code == code, gs
+    with pytest.raises(mq.MlxqError) as e:
+        mq.mlxq_quantize(0, handle(16), 0)
+    assert e.value.code == mq.MLXQ_ERR_INVALID_ARG
+    with pytest.raises(mq.MlxqError) as e:   # the codes would overwrite the source
+        mq.mlxq_quantize(base + 16, handle(16), 0)
+    assert e.value.code == mq.MLXQ_ERR_INVALID_ARG and "overlap" in mq.mlxq_last_error()
+    mq.mlxq_quantize(w, mq.mlxq_weight(base, base + 4096, base + 8192, 0, K, 16), 0)  # N = 0: no work

@@ -274,6 +274,63 @@ def test_fused_mlp_chain_concatenated_gate_up():
     assert_close(host_bits(y2), oracle.silu_gate_resid(*Wd.host, gs, gub[:F], gub[F:], xr), "down after concatenated gate/up")
 
 
+# ---------------------------------------------------------------- quantize
+QUANT_SHAPES = [(256, 512, 64), (300, 1040, 16), (77, 2048, 32), (1, 64, 64), (128, 4096, 128), (5, 24, 4),
+                (64, 512, 8), (16, 1024, 256), (33, 768, 48)]
+
+
+def run_quantize(w_bits, gs, offset_elems=0):
+    N, K = w_bits.shape
+    src = torch.zeros(N * K + offset_elems, dtype=torch.int16, device="cuda")
+    src[offset_elems:] = torch.from_numpy(w_bits.view(np.int16).ravel()).cuda()
+    packed = torch.empty((N, K // 4), dtype=torch.int32, device="cuda")
+    scales = torch.empty((N, K // gs), dtype=torch.int16, device="cuda")
+    biases = torch.empty((N, K // gs), dtype=torch.int16, device="cuda")
+    dst = mq.weight_view(packed, scales, biases, gs)
+    mq.mlxq_quantize(src.data_ptr() + 2 * offset_elems, dst)
+    torch.cuda.synchronize()
+    return (packed.cpu().numpy().view(np.uint32), scales.cpu().numpy().view(np.uint16),
+            biases.cpu().numpy().view(np.uint16)), (packed, scales, biases, dst)
+
+
+@pytest.mark.parametrize("N,K,gs", QUANT_SHAPES)
+def test_quantize_bit_exact(N, K, gs):
+    g = synth.rng(60)
+    w = synth.to_bf16_bits((g.standard_normal((N, K)) * 0.04).astype(np.float32))
+    want = oracle.quantize(w, gs)
+    for off in (0, 1):  # 8-byte loads, and a source that only allows 2-byte loads
+        got, _ = run_quantize(w, gs, off)
+        for a, b, what in zip(got, want, ("codes", "scales", "biases")):
+            assert np.array_equal(a, b), f"{what} {N}x{K}/{gs} offset {off}"
+
+
+def test_quantize_then_gemv():
+    # the quantised weight goes straight into the other calls
+    g = synth.rng(61)
+    N, K, gs = 512, 2048, 64
+    w = synth.to_bf16_bits((g.standard_normal((N, K)) * 0.05).astype(np.float32))
+    host, (_, _, _, dst) = run_quantize(w, gs)
+    x = synth.activations(g, K)
+    y = torch.empty(N, dtype=torch.bfloat16, device="cuda")
+    mq.mlxq_gemv(dst, dev(x), y)
+    torch.cuda.synchronize()
+    assert_close(host_bits(y), oracle.gemv(*host, gs, x), "gemv of a quantised weight")
+
+
+def test_quantize_constant_and_signed_zero_groups():
+    # range 0 (scale 0, codes 0) and groups of signed zeros: the first
+    # minimum in column order decides the bias's sign, as in the oracle
+    N, K, gs = 4, 64, 16
+    w = np.zeros((N, K), np.uint16)
+    w[0, :16] = 0x3EC0            # 0.375
+    w[1, 16:32:2] = 0x8000        # -0 then +0 alternating
+    w[2, 33:48:2] = 0x8000        # +0 first, then -0
+    w[3] = synth.to_bf16_bits(np.linspace(-1, 1, K).astype(np.float32))
+    got, _ = run_quantize(w, gs)
+    for a, b in zip(got, oracle.quantize(w, gs)):
+        assert np.array_equal(a, b)
+
+
 # ---------------------------------------------------------------- gemm
 def run_gemm(W, X_bits, m, kernel=mq.MLXQ_GEMM_AUTO):
     X = dev(X_bits)

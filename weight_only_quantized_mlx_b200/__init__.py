@@ -38,7 +38,8 @@ MLXQ_GEMM_SMALLM_FFMA = 4
 
 EXPORTS = ("mlxq_load", "mlxq_dequant", "mlxq_gemv", "mlxq_gemv_silu_gate",
            "mlxq_gemv_silu_gate_resid", "mlxq_gemm", "mlxq_gemm_with", "mlxq_gemm_noalloc", "mlxq_release",
-           "mlxq_last_error", "mlxq_device_status", "mlxq_selftest_wait_timeout", "mlxq_selftest_fail_alloc")
+           "mlxq_last_error", "mlxq_device_status", "mlxq_quantize", "mlxq_selftest_wait_timeout",
+           "mlxq_selftest_fail_alloc")
 
 
 class mlxq_weight(ctypes.Structure):
@@ -77,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "mlxq_release": [W],
             "mlxq_last_error": [],
             "mlxq_device_status": [],
+            "mlxq_quantize": [vp, W, u64],
             "mlxq_selftest_wait_timeout": [u32, u64],
             "mlxq_selftest_fail_alloc": [u32],
         }
@@ -158,6 +160,10 @@ MLXQ_STATIC_SCRATCH_BYTES = 40 << 20
 
 def mlxq_device_status() -> None:
     _check(lib().mlxq_device_status())
+
+
+def mlxq_quantize(w_bf16, dst: mlxq_weight, stream=None) -> None:
+    _check(lib().mlxq_quantize(_ptr(w_bf16), ctypes.byref(dst), _stream(stream)))
 
 
 def mlxq_selftest_wait_timeout(limit_us: int, stream=None) -> None:

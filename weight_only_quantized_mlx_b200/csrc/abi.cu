@@ -423,6 +423,22 @@ extern "C" {
 
 const char* mlxq_last_error(void) { return g_err.c_str(); }
 
+int mlxq_quantize(const void* w_bf16, const mlxq_weight* dst, uint64_t stream) {
+    WeightView v;
+    int rc = check_weight(dst, v);
+    if (rc) return rc;
+    if (v.gs % 4 != 0)
+        return fail(MLXQ_ERR_UNSUPPORTED, "quantize needs group_size %% 4 == 0 (got %lld)", static_cast<long long>(v.gs));
+    if ((rc = check_buf(w_bf16, v.N * v.K, "w"))) return rc;
+    const int64_t wbytes = v.N * v.K * 2, pbytes = v.N * v.K, tbytes = v.N * v.G * 2;
+    if (overlap(w_bf16, wbytes, v.packed, pbytes) || overlap(w_bf16, wbytes, v.scales, tbytes) ||
+        overlap(w_bf16, wbytes, v.biases, tbytes) || overlap(v.packed, pbytes, v.scales, tbytes) ||
+        overlap(v.packed, pbytes, v.biases, tbytes) || overlap(v.scales, tbytes, v.biases, tbytes))
+        return fail(MLXQ_ERR_INVALID_ARG, "quantize source and destination buffers overlap");
+    if (v.N == 0 || v.K == 0) return ok();
+    return launch_status(launch_quantize(w_bf16, v, as_stream(stream)), "quantize launch");
+}
+
 int mlxq_selftest_fail_alloc(uint32_t nth) {
     g_fail_alloc_in.store(static_cast<int>(nth > 1000000u ? 1000000u : nth));
     return ok();

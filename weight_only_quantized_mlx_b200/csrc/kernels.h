@@ -93,6 +93,9 @@ cudaError_t launch_gemm_smallm(const WeightView& w, const void* X, void* Y, int6
 
 // tcgen05 tensor-core gemm.
 bool gemm_tc_supported(const WeightView& w, int64_t m, const void* X, const void* Y);
+// BF16 W [N, K] (row-major) -> codes, scales and biases of `dst`.
+cudaError_t launch_quantize(const void* w, const WeightView& dst, cudaStream_t stream);
+
 // Self-test: one bounded wait that runs out after limit_ns (status word set).
 cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream);
 
