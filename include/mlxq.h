@@ -165,6 +165,22 @@ enum {
 MLXQ_API int mlxq_gemm_with(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kernel,
                    uint64_t stream);
 
+/* Output formats of mlxq_dequant_as. */
+enum { MLXQ_DTYPE_BF16 = 0, MLXQ_DTYPE_F16 = 1, MLXQ_DTYPE_F32 = 2 };
+
+/*
+ * mlxq_dequant_as (dequantize_to in another format; the dequantize-to-f16
+ * and -f32 variants of the quantized-storage page).  Writes the full
+ * weight, row-major [N, K], to out (N * K elements of the format, aligned to
+ * its size):
+ *   MLXQ_DTYPE_BF16  exactly mlxq_dequant;
+ *   MLXQ_DTYPE_F32   fma_f32(s, q, b) itself (no further rounding);
+ *   MLXQ_DTYPE_F16   fma_f32(s, q, b) rounded to FP16, nearest even.
+ * MLXQ_ERR_INVALID_ARG for an unknown dtype or a null/misaligned/overlapping
+ * out.
+ */
+MLXQ_API int mlxq_dequant_as(const mlxq_weight* w, void* out, int dtype, uint64_t stream);
+
 /*
  * mlxq_quantize (no page entry: the inverse of the format; the pages give no
  * quantizer algorithm, so the plain per-group min/max affine one is used).

@@ -152,6 +152,11 @@ class Oracle:
                                _p(scales, ctypes.c_uint16), _p(biases, ctypes.c_uint16))
         return packed, scales, biases
 
+    def dequant_f16(self, packed, scales, biases, gs) -> np.ndarray:
+        """FP16 bit patterns of fma_f32(s, q, b) rounded to nearest even (the
+        fp32 -> fp16 step is numpy's IEEE conversion), [N, K]."""
+        return self.dequant_f32(packed, scales, biases, gs).astype(np.float16).view(np.uint16)
+
     def dequant(self, packed, scales, biases, gs) -> np.ndarray:
         """BF16 bit patterns of the dequantised weight, [N, K] row-major."""
         args, keep, N, K = self._weight(packed, scales, biases, gs)

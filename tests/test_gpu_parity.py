@@ -274,6 +274,27 @@ def test_fused_mlp_chain_concatenated_gate_up():
     assert_close(host_bits(y2), oracle.silu_gate_resid(*Wd.host, gs, gub[:F], gub[F:], xr), "down after concatenated gate/up")
 
 
+# ---------------------------------------------------------------- dequant to FP16 / FP32
+@pytest.mark.parametrize("N,K,gs", [(256, 512, 64), (37, 1040, 16), (9, 60, 12), (4096, 4096, 64)])
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_dequant_as_bit_exact(N, K, gs, dtype):
+    W, _ = make(70, N, K, gs)
+    code, tdt, want = {"f16": (mq.MLXQ_DTYPE_F16, torch.float16, oracle.dequant_f16),
+                       "f32": (mq.MLXQ_DTYPE_F32, torch.float32, oracle.dequant_f32)}[dtype]
+    ref = want(*W.host, gs)
+    for off in (0, 1):  # vector stores, and an output aligned only to its element
+        buf = torch.empty(N * K + off, dtype=tdt, device="cuda")
+        mq.mlxq_dequant_as(W.w, buf.data_ptr() + off * buf.element_size(), code)
+        torch.cuda.synchronize()
+        got = buf[off:].cpu().numpy().reshape(N, K)
+        assert np.array_equal(got.view(np.uint16 if dtype == "f16" else np.uint32),
+                              ref.view(np.uint16 if dtype == "f16" else np.uint32)), (dtype, off)
+    out = torch.empty(N * K, dtype=torch.bfloat16, device="cuda")
+    mq.mlxq_dequant_as(W.w, out, mq.MLXQ_DTYPE_BF16)  # BF16: the page's dequantize_to
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(out), oracle.dequant(*W.host, gs).ravel())
+
+
 # ---------------------------------------------------------------- quantize
 QUANT_SHAPES = [(256, 512, 64), (300, 1040, 16), (77, 2048, 32), (1, 64, 64), (128, 4096, 128), (5, 24, 4),
                 (64, 512, 8), (16, 1024, 256), (33, 768, 48)]

@@ -349,11 +349,23 @@ def pin_quantize_constant_group(o: Oracle):
     assert np.array_equal(o.dequant(p, s, b, 16), w)
 
 
+def pin_dequant_f16(o: Oracle):
+    # s = 1, b = 0: codes 0..255 are exact in FP16.  s = 1, b = 2048: 2048 + q
+    # needs 12 bits, so odd q rounds to even: 2049 -> 2048, 2051 -> 2052.
+    q = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    ones = np.full((1, 4), 0x3F80, np.uint16)
+    w = o.dequant_f16(pack_le(q), ones, np.zeros((1, 4), np.uint16), 64)
+    assert np.array_equal(w.view(np.float16).astype(np.float64), q.astype(np.float64))
+    b2048 = np.full((1, 4), 0x4500, np.uint16)  # 2048 in BF16
+    w = o.dequant_f16(pack_le(q), ones, b2048, 64).view(np.float16).astype(np.float64)[0]
+    assert w[1] == 2048 and w[3] == 2052 and w[2] == 2050 and w[255] == 2048 + 256
+
+
 PINS = [pin_bf16_f32_table, pin_bf16_f64_table, pin_bf16_two_routes_agree, pin_unpack_word,
         pin_identity_scale, pin_centred_scale, pin_group_index, pin_worked_example,
         pin_bruteforce, pin_integer_exact, pin_silu_closed_forms, pin_silu_gate_zero,
         pin_silu_gate_structure, pin_gemm_rows_are_gemv, pin_quantize_grid_identity,
-        pin_quantize_error_bound, pin_quantize_constant_group]
+        pin_quantize_error_bound, pin_quantize_constant_group, pin_dequant_f16]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)

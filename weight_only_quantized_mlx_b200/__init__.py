@@ -36,9 +36,13 @@ MLXQ_GEMM_SMALLM = 2
 MLXQ_GEMM_TCGEN05 = 3
 MLXQ_GEMM_SMALLM_FFMA = 4
 
+MLXQ_DTYPE_BF16 = 0
+MLXQ_DTYPE_F16 = 1
+MLXQ_DTYPE_F32 = 2
+
 EXPORTS = ("mlxq_load", "mlxq_dequant", "mlxq_gemv", "mlxq_gemv_silu_gate",
            "mlxq_gemv_silu_gate_resid", "mlxq_gemm", "mlxq_gemm_with", "mlxq_gemm_noalloc", "mlxq_release",
-           "mlxq_last_error", "mlxq_device_status", "mlxq_quantize", "mlxq_selftest_wait_timeout",
+           "mlxq_last_error", "mlxq_device_status", "mlxq_dequant_as", "mlxq_quantize", "mlxq_selftest_wait_timeout",
            "mlxq_selftest_fail_alloc")
 
 
@@ -79,6 +83,7 @@ def lib() -> ctypes.CDLL:
             "mlxq_last_error": [],
             "mlxq_device_status": [],
             "mlxq_quantize": [vp, W, u64],
+            "mlxq_dequant_as": [W, vp, i32, u64],
             "mlxq_selftest_wait_timeout": [u32, u64],
             "mlxq_selftest_fail_alloc": [u32],
         }
@@ -160,6 +165,10 @@ MLXQ_STATIC_SCRATCH_BYTES = 40 << 20
 
 def mlxq_device_status() -> None:
     _check(lib().mlxq_device_status())
+
+
+def mlxq_dequant_as(w: mlxq_weight, out, dtype: int, stream=None) -> None:
+    _check(lib().mlxq_dequant_as(ctypes.byref(w), _ptr(out), dtype, _stream(stream)))
 
 
 def mlxq_quantize(w_bf16, dst: mlxq_weight, stream=None) -> None:

@@ -526,6 +526,21 @@ int mlxq_dequant(const mlxq_weight* w, void* out, uint64_t stream) {
     return launch_status(launch_dequant(v, out, as_stream(stream)), "mlx_int8_dequant launch");
 }
 
+int mlxq_dequant_as(const mlxq_weight* w, void* out, int dtype, uint64_t stream) {
+    WeightView v;
+    int rc = check_weight(w, v);
+    if (rc) return rc;
+    if (dtype < MLXQ_DTYPE_BF16 || dtype > MLXQ_DTYPE_F32) return fail(MLXQ_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+    const int64_t esize = dtype == MLXQ_DTYPE_F32 ? 4 : 2;
+    if (v.N * v.K != 0) {
+        if (!out) return fail(MLXQ_ERR_INVALID_ARG, "out is null");
+        if (!aligned(out, static_cast<size_t>(esize))) return fail(MLXQ_ERR_INVALID_ARG, "out is not %lld-byte aligned",
+                                                                    static_cast<long long>(esize));
+    }
+    if ((rc = check_out_vs_weight(out, v.N * v.K * esize, v))) return rc;
+    return launch_status(launch_dequant_as(v, out, dtype, as_stream(stream)), "dequant launch");
+}
+
 static int gemv_common(const mlxq_weight* w, int mode, const void* x, const void* gate, const void* up,
                        const void* resid, void* y, uint64_t stream) {
     WeightView v;

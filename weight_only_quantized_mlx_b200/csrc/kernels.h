@@ -72,6 +72,8 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 // mlx_int8_dequant: out [N, K] bf16.
 cudaError_t launch_dequant(const WeightView& w, void* out, cudaStream_t stream);
+// dtype: 0 BF16 (launch_dequant), 1 FP16, 2 FP32.
+cudaError_t launch_dequant_as(const WeightView& w, void* out, int dtype, cudaStream_t stream);
 
 // mlx_int8_gemv family (m = 1): y = W h (+ resid), h = x or silu(gate)*up.
 cudaError_t launch_gemv(const WeightView& w, int mode, const void* x, const void* gate,
