@@ -291,3 +291,19 @@ def test_quantize_validation_before_any_launch():
         mq.mlxq_quantize(base + 16, handle(16), 0)
     assert e.value.code == mq.MLXQ_ERR_INVALID_ARG and "overlap" in mq.mlxq_last_error()
     mq.mlxq_quantize(w, mq.mlxq_weight(base, base + 4096, base + 8192, 0, K, 16), 0)  # N = 0: no work
+
+
+def test_weight_dimensions_beyond_any_device_are_rejected():
+    base = 1 << 40
+    w = mq.mlxq_weight(base, base + 4096, base + 8192, 0xFFFFFFF0, 0xFFFFFFF0, 16)
+    with pytest.raises(mq.MlxqError) as e:
+        mq.mlxq_dequant(w, base + (1 << 20), 0)
+    assert e.value.code == mq.MLXQ_ERR_SHAPE
+
+
+def test_gemm_rows_beyond_any_device_are_rejected():
+    base = 1 << 40
+    w = mq.mlxq_weight(base, base + (1 << 30), base + (2 << 30), 4096, 1 << 24, 64)
+    with pytest.raises(mq.MlxqError) as e:
+        mq.mlxq_gemm(w, base + (3 << 30), base + (4 << 30), 0xFFFFFFFF, 0)
+    assert e.value.code == mq.MLXQ_ERR_SHAPE

@@ -339,6 +339,11 @@ int check_weight(const mlxq_weight* w, WeightView& v) {
                     w->in_features);
     if (!aligned(w->packed, 4) || !aligned(w->scales, 2) || !aligned(w->biases, 2))
         return fail(MLXQ_ERR_INVALID_ARG, "weight buffers are misaligned");
+    // every byte count below (up to 4 bytes per weight, times m for gemm
+    // outputs checked separately) must stay far inside int64
+    if (static_cast<uint64_t>(w->out_features) * w->in_features > (1ull << 50))
+        return fail(MLXQ_ERR_SHAPE, "out_features x in_features = %llu is beyond any device",
+                    static_cast<unsigned long long>(static_cast<uint64_t>(w->out_features) * w->in_features));
     v.packed = static_cast<const uint32_t*>(w->packed);
     v.scales = static_cast<const uint16_t*>(w->scales);
     v.biases = static_cast<const uint16_t*>(w->biases);
@@ -591,6 +596,8 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
         return fail(MLXQ_ERR_INVALID_ARG, "unknown gemm kernel id %d", kernel);
     if (m == 0) return ok();
     const int64_t M = m;
+    if ((v.K > v.N ? v.K : v.N) > (int64_t{1} << 50) / M)
+        return fail(MLXQ_ERR_SHAPE, "m x in_features or m x out_features is beyond any device");
     if ((rc = check_buf(x, M * v.K, "X"))) return rc;
     if ((rc = check_buf(y, M * v.N, "Y"))) return rc;
     if (overlap(y, M * v.N * 2, x, M * v.K * 2)) return fail(MLXQ_ERR_INVALID_ARG, "Y overlaps X");
