@@ -307,3 +307,18 @@ def test_gemm_rows_beyond_any_device_are_rejected():
     with pytest.raises(mq.MlxqError) as e:
         mq.mlxq_gemm(w, base + (3 << 30), base + (4 << 30), 0xFFFFFFFF, 0)
     assert e.value.code == mq.MLXQ_ERR_SHAPE
+
+
+def test_public_header_is_plain_c99(tmp_path):
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "mlxq.h"\n'
+                   "int main(void) { mlxq_weight w = {0}; (void)w;\n"
+                   "  return MLXQ_OK + MLXQ_DTYPE_F32 + MLXQ_GEMM_TCGEN05 - 5; }\n")
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, "-c", str(src),
+                        "-o", str(tmp_path / "use_header.o")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
