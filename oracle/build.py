@@ -1,6 +1,6 @@
 """Compile the CPU oracle (plain single-threaded C++) into oracle/libmlxq_oracle.so.
 
-Test infrastructure: the library this builds is the independent checker of the
+Test infrastructure: the library built here is the independent checker of the
 CUDA path and is loaded only by the tests, the smoke check and the benchmark's
 CPU-baseline leg.
 """

@@ -27,7 +27,7 @@
 //     reading below is pinned by invariants only (grid identity, error bound,
 //     constant groups).
 //
-// Readings taken where the page is silent (each is listed in the design doc):
+// Readings taken where the page is silent:
 //   * q[n,k] is byte (k mod 4) of word packed[n, k/4], little-endian
 //     (byte j = bits 8j..8j+7), unsigned 0..255.
 //   * W[n,k] = bf16_rne( fma_f32(s[n,g], q[n,k], b[n,g]) ), g = floor(k/gs):
