@@ -1,4 +1,4 @@
-// TMA tensor maps (CUtensorMap) for the kernels: the driver's encoder is
+// TMA tensor maps (CUtensorMap) for the kernels: the CUDA driver's encoder is
 // reached through the CUDA runtime (no libcuda link), and the maps of a
 // weight's three buffers are cached per (buffers, shape, box) so repeated
 // calls on the same weight do not re-encode them.
