@@ -322,3 +322,22 @@ def test_public_header_is_plain_c99(tmp_path):
     r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, "-c", str(src),
                         "-o", str(tmp_path / "use_header.o")], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_dequant_as_validation_before_any_launch():
+    base = 1 << 40
+    w = mq.mlxq_weight(base, base + (1 << 20), base + (2 << 20), 16, 64, 16)
+    out = base + (3 << 20)
+    for bad_dtype in (-1, 3):
+        with pytest.raises(mq.MlxqError) as e:
+            mq.mlxq_dequant_as(w, out, bad_dtype, 0)
+        assert e.value.code == mq.MLXQ_ERR_INVALID_ARG
+    with pytest.raises(mq.MlxqError) as e:      # FP32 output must be 4-byte aligned
+        mq.mlxq_dequant_as(w, out + 2, mq.MLXQ_DTYPE_F32, 0)
+    assert e.value.code == mq.MLXQ_ERR_INVALID_ARG and "aligned" in mq.mlxq_last_error()
+    with pytest.raises(mq.MlxqError) as e:
+        mq.mlxq_dequant_as(w, 0, mq.MLXQ_DTYPE_F16, 0)
+    assert e.value.code == mq.MLXQ_ERR_INVALID_ARG
+    with pytest.raises(mq.MlxqError) as e:      # output would overwrite the packed codes
+        mq.mlxq_dequant_as(w, base, mq.MLXQ_DTYPE_F32, 0)
+    assert e.value.code == mq.MLXQ_ERR_INVALID_ARG
