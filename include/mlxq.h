@@ -127,8 +127,9 @@ MLXQ_API int mlxq_gemv_silu_gate_resid(const mlxq_weight* w, const void* gate, c
  * tensor-core kernel for larger m (weight tiles dequantised to BF16 in shared
  * memory, fp32 accumulators in TMEM).  When m leaves SMs idle, the
  * tensor-core kernel splits K over CTAs; their fp32 partials live in a
- * stream-ordered memory pool owned by the library (allocated and freed on
- * `stream`, so the call can be captured in a CUDA graph).
+ * stream-ordered memory pool owned by the library, allocated and freed in
+ * order on `stream`.  To capture such a call in a CUDA graph, use
+ * mlxq_gemm_noalloc, which allocates nothing (tested inside a graph).
  */
 MLXQ_API int mlxq_gemm(const mlxq_weight* w, const void* x, void* y, uint32_t m, uint64_t stream);
 
