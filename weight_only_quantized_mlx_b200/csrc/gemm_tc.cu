@@ -685,7 +685,7 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
         return cudaGetLastError();
     }
     // K split: the fp32 partials and the per-tile counters come from the
-    // stream-ordered pool (so the call also works under graph capture)
+    // library's stream-ordered pool, allocated and freed in order on the stream
     const size_t bytes = part_bytes + static_cast<size_t>(tiles) * sizeof(unsigned int);
     cudaMemPool_t pool;
     e = workspace_pool(dev.device, &pool);
