@@ -563,9 +563,9 @@ cudaError_t static_scratch_base(int device, unsigned char** out) {
     return cudaSuccess;
 }
 
-// Synchronous: called from mlxq_device_status after a device-wide sync.
 }  // namespace
 
+// Synchronous: called from mlxq_device_status after a device-wide sync.
 cudaError_t reset_static_scratch_counters() {
     const DeviceInfo& dev = device_info();
     unsigned char* base = nullptr;
