@@ -34,11 +34,13 @@ def _signatures():
     return {
         "oracle_bf16_from_f32": (ctypes.c_uint16, [ctypes.c_float]),
         "oracle_bf16_from_f64": (ctypes.c_uint16, [ctypes.c_double]),
+        "oracle_f16_from_f32": (ctypes.c_uint16, [ctypes.c_float]),
         "oracle_f32_from_bf16": (ctypes.c_float, [ctypes.c_uint16]),
         "oracle_silu": (ctypes.c_double, [ctypes.c_double]),
         "oracle_unpack": (None, [u32p, i64, i64, u8p]),
         "oracle_dequant_f32": (None, W + [f32p]),
         "oracle_dequant": (None, W + [u16p]),
+        "oracle_dequant_f16": (None, W + [u16p]),
         "oracle_gemv_f64": (None, W + [u16p, f64p]),
         "oracle_gemv": (None, W + [u16p, u16p]),
         "oracle_silu_gate_f64": (None, W + [u16p, u16p, f64p]),
@@ -153,9 +155,14 @@ class Oracle:
         return packed, scales, biases
 
     def dequant_f16(self, packed, scales, biases, gs) -> np.ndarray:
-        """FP16 bit patterns of fma_f32(s, q, b) rounded to nearest even (the
-        fp32 -> fp16 step is numpy's IEEE conversion), [N, K]."""
-        return self.dequant_f32(packed, scales, biases, gs).astype(np.float16).view(np.uint16)
+        """FP16 bit patterns of fma_f32(s, q, b) rounded to nearest even, [N, K]."""
+        args, keep, N, K = self._weight(packed, scales, biases, gs)
+        w = np.empty((N, K), np.uint16)
+        self.L.oracle_dequant_f16(*args, _p(w, ctypes.c_uint16))
+        return w
+
+    def f16_from_f32(self, v: float) -> int:
+        return int(self.L.oracle_f16_from_f32(float(v)))
 
     def dequant(self, packed, scales, biases, gs) -> np.ndarray:
         """BF16 bit patterns of the dequantised weight, [N, K] row-major."""

@@ -16,7 +16,9 @@
 //     [out_features, in_features/4] bytes held in uint32 words; scales and
 //     biases are [out_features, in_features/group_size] BF16, one per group.
 //   * "load": group_size must divide in_features.
-//   * "dequantize_to": the full dequantised weight, BF16.
+//   * "dequantize_to": the full dequantised weight, BF16.  The
+//     quantized-storage page also names dequantisation to f16 and f32: the
+//     fp32 affine value itself, and that value rounded to FP16 (nearest even).
 //   * "gemv": y = W x.
 //   * "gemv_silu_gate": y = W (silu(gate) * up).
 //   * "gemv_silu_gate_resid": y[n] = x_resid[n] + sum_k W[n,k]*(silu(gate[k])*up[k]).
@@ -86,6 +88,39 @@ uint16_t f64_to_bf16(double v) {
     return static_cast<uint16_t>(u >> 16);
 }
 
+// ---- FP16 (IEEE binary16: 1 sign, 5 exponent, 10 stored significand bits) --
+
+// fp32 -> fp16, round to nearest, ties to even, written on the fp32 bit
+// pattern.  A finite fp32 value is sig * 2^(E - 23) with a 24-bit integer
+// significand sig (implicit bit included for normal numbers).  Its fp16
+// quantum is 2^(max(E, -14) - 10): 10 fraction bits for normal numbers, the
+// fixed subnormal step 2^-24 below 2^-14.  The dropped low bits of sig decide
+// the rounding (above half: up; exactly half: to the even neighbour).  A carry
+// out of the significand moves into the exponent field by itself, so the
+// largest subnormal rounds up to the smallest normal and 65520 and above
+// overflow to infinity.  NaN stays NaN (quiet bit set, top payload bits kept).
+uint16_t f32_to_f16(float v) {
+    uint32_t u;
+    std::memcpy(&u, &v, 4);
+    const uint16_t sign = static_cast<uint16_t>((u >> 16) & 0x8000u);
+    const uint32_t a = u & 0x7FFFFFFFu;
+    if (a > 0x7F800000u) return static_cast<uint16_t>(sign | 0x7E00u | ((a >> 13) & 0x3FFu));
+    if (a == 0x7F800000u) return static_cast<uint16_t>(sign | 0x7C00u);
+    const int biased = static_cast<int>(a >> 23);
+    const uint32_t sig = biased == 0 ? (a & 0x7FFFFFu) : ((a & 0x7FFFFFu) | 0x800000u);
+    const int E = biased == 0 ? -126 : biased - 127;
+    if (E > 15) return static_cast<uint16_t>(sign | 0x7C00u);  // |v| >= 2^16
+    const int qe = (E < -14 ? -14 : E) - 10;                   // fp16 quantum 2^qe
+    const int shift = qe - (E - 23);                           // dropped bits, >= 13
+    if (shift > 24) return sign;  // |v| < 2^-25: below half the smallest subnormal
+    uint32_t mant = sig >> shift;
+    const uint32_t rem = sig & ((1u << shift) - 1u);
+    const uint32_t half = 1u << (shift - 1);
+    if (rem > half || (rem == half && (mant & 1u))) mant += 1u;
+    const uint32_t bits = (static_cast<uint32_t>((E < -14 ? -14 : E) + 14) << 10) + mant;
+    return static_cast<uint16_t>(sign | (bits >= 0x7C00u ? 0x7C00u : bits));
+}
+
 float bf16_to_f32(uint16_t h) {
     const uint32_t u = static_cast<uint32_t>(h) << 16;
     float f;
@@ -132,6 +167,7 @@ extern "C" {
 // ---- scalar conversions (exposed so the tests can pin them) ---------------
 uint16_t oracle_bf16_from_f32(float v) { return f32_to_bf16(v); }
 uint16_t oracle_bf16_from_f64(double v) { return f64_to_bf16(v); }
+uint16_t oracle_f16_from_f32(float v) { return f32_to_f16(v); }
 float oracle_f32_from_bf16(uint16_t h) { return bf16_to_f32(h); }
 double oracle_silu(double t) { return silu_f64(t); }
 
@@ -150,6 +186,15 @@ void oracle_dequant_f32(const uint32_t* packed, const uint16_t* scales,
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k)
             w[n * K + k] = affine_f32(packed, scales, biases, K, gs, n, k);
+}
+
+// fp32 affine values rounded to FP16 (nearest even), as bit patterns.
+void oracle_dequant_f16(const uint32_t* packed, const uint16_t* scales,
+                        const uint16_t* biases, int64_t N, int64_t K, int64_t gs,
+                        uint16_t* w) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            w[n * K + k] = f32_to_f16(affine_f32(packed, scales, biases, K, gs, n, k));
 }
 
 // The BF16 weight, row-major [N, K], as bit patterns.

@@ -349,6 +349,35 @@ def pin_quantize_constant_group(o: Oracle):
     assert np.array_equal(o.dequant(p, s, b, 16), w)
 
 
+def pin_f16_f32_table(o: Oracle):
+    for line in open(os.path.join(GOLDEN, "fp16_rne_f32.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        f_hex, h_hex = line.split()[:2]
+        v = np.array([int(f_hex, 16)], np.uint32).view(np.float32)[0]
+        got = o.f16_from_f32(v)
+        assert got == int(h_hex, 16), f"{f_hex}: got {got:04X}, want {h_hex}"
+
+
+def pin_f16_matches_ieee_conversion(o: Oracle):
+    # The same rule, implemented independently by numpy's IEEE float32 ->
+    # float16 conversion, on random values across the normal, subnormal,
+    # overflow and tie ranges.
+    g = np.random.default_rng(11)
+    vals = np.concatenate([
+        g.standard_normal(4000).astype(np.float32),
+        (g.standard_normal(2000) * 2.0 ** -18).astype(np.float32),     # subnormal FP16 range
+        (g.uniform(6.0e4, 7.0e4, 1000) * g.choice([-1, 1], 1000)).astype(np.float32),  # overflow edge
+        ((g.integers(-2048, 2048, 2000) + 0.5) * 2.0 ** -10).astype(np.float32),      # exact ties
+    ])
+    with np.errstate(over="ignore"):
+        want = vals.astype(np.float16).view(np.uint16)
+    got = np.array([o.f16_from_f32(v) for v in vals], np.uint16)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, f"{bad.size} mismatches, first {vals[bad[0]]!r}: {got[bad[0]]:04X} vs {want[bad[0]]:04X}"
+
+
 def pin_dequant_f16(o: Oracle):
     # s = 1, b = 0: codes 0..255 are exact in FP16.  s = 1, b = 2048: 2048 + q
     # needs 12 bits, so odd q rounds to even: 2049 -> 2048, 2051 -> 2052.
@@ -365,7 +394,8 @@ PINS = [pin_bf16_f32_table, pin_bf16_f64_table, pin_bf16_two_routes_agree, pin_u
         pin_identity_scale, pin_centred_scale, pin_group_index, pin_worked_example,
         pin_bruteforce, pin_integer_exact, pin_silu_closed_forms, pin_silu_gate_zero,
         pin_silu_gate_structure, pin_gemm_rows_are_gemv, pin_quantize_grid_identity,
-        pin_quantize_error_bound, pin_quantize_constant_group, pin_dequant_f16]
+        pin_quantize_error_bound, pin_quantize_constant_group, pin_dequant_f16, pin_f16_f32_table,
+        pin_f16_matches_ieee_conversion]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -391,6 +421,8 @@ MUTANTS = {
     "quant_divisor_256": ("f32_to_bf16(range / 255.0f)", "f32_to_bf16(range / 256.0f)"),
     "quant_bias_from_max": ("const uint16_t bb = f32_to_bf16(lo);", "const uint16_t bb = f32_to_bf16(hi);"),
     "quant_round_down": ("c = std::nearbyint(d / sf);", "c = std::floor(d / sf);"),
+    "f16_ties_away": ("(rem == half && (mant & 1u))", "(rem == half)"),
+    "f16_no_subnormals": ("if (shift > 24) return sign;", "if (E < -14) return sign;"),
 }
 
 
