@@ -55,17 +55,23 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def profile_traffic(kernel_tag: str, source_files):
-    """dram bytes per launch from a committed ncu summary, or None when the
-    summary is missing or the kernel sources changed since it was taken."""
+def source_hash(source_files, root=ROOT) -> str:
+    """First 16 hex digits of the sha256 over the given files' bytes, in order."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
-    if not os.path.exists(path):
-        return None
     h = hashlib.sha256()
     for f in source_files:
-        with open(os.path.join(ROOT, f), "rb") as fh:
+        with open(os.path.join(root, f), "rb") as fh:
             h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel_tag: str, source_files, root=ROOT):
+    """dram bytes per launch from a committed ncu summary, or None when the
+    summary is missing or the kernel sources changed since it was taken."""
+    path = os.path.join(root, "profiles", f"{kernel_tag}.md")
+    if not os.path.exists(path):
+        return None
+    digest = source_hash(source_files, root)
     vals = {}
     for line in open(path):
         if ":" in line and line.strip().startswith("- "):
@@ -74,7 +80,7 @@ def profile_traffic(kernel_tag: str, source_files):
             if v.startswith("`") and v.count("`") >= 2:
                 v = v[1:v.index("`", 1)]  # the first backticked token
             vals[k.strip()] = v
-    if vals.get("source_sha256") != h.hexdigest()[:16]:
+    if vals.get("source_sha256") != digest:
         return None
     try:
         return float(vals["traffic_bytes_per_launch"])
@@ -329,17 +335,19 @@ def measure_rows(mq, torch, synth, dev, stream, dec_weights, peaks, args):
     warm = max(3, args.warmup)
     hbm = peaks["hbm_gbs"]
 
-    # dequantize_to over the 100 decode weights
-    out = torch.empty(D_N * D_K, dtype=torch.bfloat16, device=dev)
+    # dequantize_to over the 100 decode weights; the outputs rotate over 8
+    # buffers (268 MB, more than L2) so the writes reach HBM
+    outs = [torch.empty(D_N * D_K, dtype=torch.bfloat16, device=dev) for _ in range(8)]
 
     def deq():
-        for w in dec_weights:
-            mq.mlxq_dequant(w.handle, out, stream)
+        for i, w in enumerate(dec_weights):
+            mq.mlxq_dequant(w.handle, outs[i % len(outs)], stream)
     ms = time_region(deq, steps, warm, stream, 1)
     b = (D_N * D_K + 4 * D_N * D_K // D_GS + 2 * D_N * D_K) * len(dec_weights)
     gbs = b / (ms * 1e-3) / 1e9
     rows["dequant_4096x4096"] = {"value": round(gbs, 1), "unit": "GB/s", "frac_hbm": round(gbs / hbm, 4),
-                                 "bytes_per_launch": b // len(dec_weights)}
+                                 "bytes_per_launch": b // len(dec_weights), "output_buffers": len(outs)}
+    del outs
 
     # quantize: BF16 [4096, 4096] -> codes + tables, 8 sources rotating (268 MB)
     qsrc = [torch.randn(D_N, D_K, device=dev).to(torch.bfloat16) * 0.04 for _ in range(8)]
@@ -411,26 +419,30 @@ def measure_rows(mq, torch, synth, dev, stream, dec_weights, peaks, args):
         for w in ws:
             w.release()
 
-    # small-m batched decode: (N, K) in {(28672, 8192), (8192, 28672)}, gs = 64
-    for (N, K) in ((28672, 8192), (8192, 28672)):
-        w = upload_weight(mq, *synth.weight(synth.rng(3000 + N), N, K, 64), 64)
-        for m in (1, 2, 4, 8, 16, 32):
-            X = torch.randn(m, K, device=dev).to(torch.bfloat16)
-            Y = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
-            ms = time_region(lambda: mq.mlxq_gemm(w.handle, X, Y, m, stream), steps, warm, stream, 1)
-            b = gemv_bytes(N, K, 64, m)
-            rows[f"smallm_{N}x{K}_m{m}"] = {"value": round(b / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
-                                            "tflops": round(2 * m * N * K / (ms * 1e-3) / 1e12, 2),
-                                            "frac_hbm": round(b / (ms * 1e-3) / 1e9 / hbm, 4),
-                                            "us": round(ms * 1e3, 2)}
-        w.release()
+    # small-m batched decode: (N, K) in {(28672, 8192), (8192, 28672)},
+    # group_size in {32, 64, 128} (each weight 235 MB, more than L2)
+    for gs_m in (64, 32, 128):
+        for (N, K) in ((28672, 8192), (8192, 28672)):
+            w = upload_weight(mq, *synth.weight(synth.rng(3000 + N + gs_m), N, K, gs_m), gs_m)
+            for m in (1, 2, 4, 8, 16, 32):
+                X = torch.randn(m, K, device=dev).to(torch.bfloat16)
+                Y = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
+                ms = time_region(lambda: mq.mlxq_gemm(w.handle, X, Y, m, stream), steps, warm, stream, 1)
+                b = gemv_bytes(N, K, gs_m, m)
+                tag = f"smallm_{N}x{K}_m{m}" + ("" if gs_m == 64 else f"_gs{gs_m}")
+                rows[tag] = {"value": round(b / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                             "tflops": round(2 * m * N * K / (ms * 1e-3) / 1e12, 2),
+                             "frac_hbm": round(b / (ms * 1e-3) / 1e9 / hbm, 4),
+                             "us": round(ms * 1e3, 2)}
+            w.release()
 
-    # prefill gemm (tensor cores): m = 4096 fills every SM with whole tiles;
-    # m = 512 and 128 have fewer tiles than SMs, so each tile's K is split
-    # (three weight copies, 183 MB, taken in turn: larger than L2)
+    # prefill gemm (tensor cores), m in {512, 2048, 4096, 8192}: m >= 2048
+    # fills every SM with whole tiles; at m = 512 there are fewer tiles than
+    # SMs, so each tile's K is split (three weight copies, 183 MB, taken in
+    # turn: larger than L2)
     for (N, K) in ((4096, 14336), (14336, 4096)):
         ws = [upload_weight(mq, *synth.weight(synth.rng(4000 + N + i), N, K, 64), 64) for i in range(3)]
-        for m in (4096, 512, 128):
+        for m in (512, 2048, 4096, 8192):
             X = torch.randn(m, K, device=dev).to(torch.bfloat16)
             Y = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
             turn = [0]
@@ -472,7 +484,20 @@ def cpu_baseline_gemv(budget_s: float = 12.0):
     gbs = gemv_bytes(D_N, D_K, D_GS) * done / t_total / 1e9
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"{done} of the {N_PAIRS} decode pairs (N=K=4096, gs=64), one oracle gemv each",
-            "host_cpus": os.cpu_count()}
+            "host_cpus": os.cpu_count(), "cpu_model": cpu_model()}
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (first 'model name' line of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def run_reference(args):
@@ -502,7 +527,8 @@ def run_reference(args):
         "config": {"workload": "decode gemv: 100 seeded (W, x) pairs, N=4096, K=4096, group_size=64, m=1",
                    "sample_pairs_per_step": per_step_pairs},
         "impl": "reference",
-        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+                         "host_cpus": os.cpu_count(), "cpu_model": cpu_model()},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)

@@ -25,7 +25,11 @@
  *   - Outputs may not overlap inputs, except y == x_resid exactly (each
  *     output element reads its own residual before its single write).  Other
  *     overlaps that the library can see are rejected with MLXQ_ERR_INVALID_ARG.
- *   - The calls allocate no device memory per call.
+ *   - Device memory: mlxq_load allocates the weight's three buffers.  When
+ *     mlxq_gemm splits K over CTAs it takes fp32 partials from a stream-ordered
+ *     pool the library owns (allocated and freed in order on `stream`); the
+ *     pool keeps its memory between calls.  No other call allocates device
+ *     memory; mlxq_gemm_noalloc is mlxq_gemm without any allocation.
  */
 #ifndef MLXQ_H
 #define MLXQ_H
@@ -128,8 +132,7 @@ MLXQ_API int mlxq_gemv_silu_gate_resid(const mlxq_weight* w, const void* gate, c
  * memory, fp32 accumulators in TMEM).  When m leaves SMs idle, the
  * tensor-core kernel splits K over CTAs; their fp32 partials live in a
  * stream-ordered memory pool owned by the library, allocated and freed in
- * order on `stream`.  To capture such a call in a CUDA graph, use
- * mlxq_gemm_noalloc, which allocates nothing (tested inside a graph).
+ * order on `stream`.  Callers that must not allocate use mlxq_gemm_noalloc.
  */
 MLXQ_API int mlxq_gemm(const mlxq_weight* w, const void* x, void* y, uint32_t m, uint64_t stream);
 
@@ -140,14 +143,24 @@ MLXQ_API int mlxq_gemm(const mlxq_weight* w, const void* x, void* y, uint32_t m,
 
 /*
  * mlxq_gemm_noalloc (page: MlxInt8Weight::gemm, kernel mlx_int8_gemm).
- * mlxq_gemm that allocates no device memory: same arguments, layout, kernel
- * choice and results (bit for bit).  Where mlxq_gemm takes the K-split
- * partials from its memory pool, this call uses the library's static scratch
- * buffer (MLXQ_STATIC_SCRATCH_BYTES, a device array that exists from the
- * moment the library's device code loads).  A call whose split would need
- * more returns MLXQ_ERR_UNSUPPORTED and launches nothing.  The buffer is one
- * per device and shared by every call, so calls that split K must not run at
- * the same time: issue them on one stream, or order them with events.
+ * mlxq_gemm that allocates no device memory, for callers that cannot call
+ * cudaMalloc or a pool allocator: code running where allocation is not
+ * allowed or not wanted (a fixed memory budget set up front, a runtime that
+ * owns all device memory itself, or a hot loop that must not reach the
+ * allocator).  Same arguments, layout, kernel choice and results (bit for
+ * bit) as mlxq_gemm.  Where mlxq_gemm takes the K-split partials from its
+ * memory pool, this call uses the library's static scratch buffer: a
+ * file-scope device array of MLXQ_STATIC_SCRATCH_BYTES that every GPU which
+ * loads the library holds until the process exits.
+ *   - A call whose split would need more than that returns
+ *     MLXQ_ERR_UNSUPPORTED and launches nothing.
+ *   - The first call on a device that splits K looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture on the device.
+ *   - The buffer is one per device and shared by every call, and it keeps
+ *     the last call's contents (each split leaves its tile counters at zero
+ *     for the next).  Calls that overlap on the GPU race on it: issue calls
+ *     that split K on one stream, or order them with events.
  */
 MLXQ_API int mlxq_gemm_noalloc(const mlxq_weight* w, const void* x, void* y, uint32_t m, uint64_t stream);
 

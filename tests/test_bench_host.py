@@ -19,9 +19,24 @@ def test_algorithmic_bytes():
     assert chain == 187_318_272
 
 
-def test_profile_traffic_only_for_the_profiled_source():
-    srcs = ["weight_only_quantized_mlx_b200/csrc/gemv_mma.cu", "weight_only_quantized_mlx_b200/csrc/device_common.cuh"]
-    t = bench.profile_traffic("gemv_decode_4096x4096_gs64", srcs)
-    assert t is not None and 17e6 < t < 19e6       # the committed capture matches the source
-    assert bench.profile_traffic("gemv_decode_4096x4096_gs64", srcs[:1]) is None  # another source: no figure
-    assert bench.profile_traffic("no_such_profile", srcs) is None
+def test_profile_traffic_only_for_the_profiled_source(tmp_path):
+    # a summary in the committed format, recorded for one source file
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    digest = bench.source_hash(["k.cu"], str(tmp_path))
+    (tmp_path / "profiles" / "k_tag.md").write_text(
+        "# k\n\n- dram__bytes_read.sum: `17.9` Mbyte\n"
+        f"- traffic_bytes_per_launch: `17864448`\n- source_sha256: `{digest}` (of k.cu)\n")
+    assert bench.profile_traffic("k_tag", ["k.cu"], str(tmp_path)) == 17864448.0
+    assert bench.profile_traffic("no_such_profile", ["k.cu"], str(tmp_path)) is None
+    src.write_text("kernel v2\n")  # the source changed since the capture: no figure
+    assert bench.profile_traffic("k_tag", ["k.cu"], str(tmp_path)) is None
+
+
+def test_committed_profiles_name_their_sources():
+    # every committed summary that feeds a bench figure records a source hash
+    for name in os.listdir(os.path.join(ROOT, "profiles")):
+        text = open(os.path.join(ROOT, "profiles", name)).read()
+        if "traffic_bytes_per_launch" in text:
+            assert "source_sha256" in text, name

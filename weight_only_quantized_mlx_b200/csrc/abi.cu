@@ -405,8 +405,10 @@ const DeviceInfo& device_info() {
         di.device = dev;
         cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
         cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        cudaDeviceGetAttribute(&di.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
         if (di.sm_count <= 0) di.sm_count = 1;
         if (di.max_smem_optin <= 0) di.max_smem_optin = 48 * 1024;
+        if (di.smem_per_sm < di.max_smem_optin) di.smem_per_sm = di.max_smem_optin;
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_status_word) == cudaSuccess) g_status_ptr[dev] = static_cast<unsigned int*>(p);
         g_dev[dev] = di;

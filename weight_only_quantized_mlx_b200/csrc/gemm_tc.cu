@@ -24,7 +24,9 @@
 // depend on which CTA finishes when.  The accumulator is D[w_row][x_row]
 // (TMEM lane = weight row), so a warp's stores of one output row of Y are 32
 // consecutive BF16 values.  All pipeline waits are bounded; no cluster
-// multicast is used.
+// multicast is used.  After a wait gives up, the producers and the MMA thread
+// issue nothing more, and before TMEM is freed and the CTA exits they wait
+// (bounded) for the copies and MMAs they already issued.
 #include <mutex>
 
 #include "device_common.cuh"
@@ -224,7 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* sbempty = sbfull + kSSB;
     uint64_t* acc_full = sbempty + kSSB;
     uint64_t* acc_empty = acc_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+    uint64_t* drain = acc_empty + 1;  // the MMA thread's last commit (teardown)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     uint32_t* last_flag = tmem_slot + 1;  // epilogue: this CTA completed the tile
     auto A_of = [&](int s) { return sbase + static_cast<uint32_t>(s) * kStageA; };
     auto X_of = [&](int s) { return x_base + static_cast<uint32_t>(s) * stage_x; };
@@ -263,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(smem_u32(acc_full), 1);
         mbar_init(smem_u32(acc_empty), kEpilogueWarps);
+        mbar_init(smem_u32(drain), 1);
         mbar_fence_init();
     }
     if (warp == 1) {
@@ -282,18 +286,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = policy_evict_last();  // each activation tile serves every weight tile
             bool ok = true;
             int it = 0;
-            for (int t = 0; t < my_units; ++t) {
+            for (int t = 0; t < my_units && ok; ++t) {
                 int tile, split, n0, m0, kb0, kb1;
                 unit_of(t, tile, split, n0, m0, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % SX;
-                    if (it >= SX && ok) ok = mbar_wait(smem_u32(&xempty[s]), ((it / SX) - 1) & 1, p.status);
+                    if (it >= SX) ok = mbar_wait(smem_u32(&xempty[s]), ((it / SX) - 1) & 1, p.status);
+                    if (!ok) break;  // the slot may still be in use: issue nothing more
                     mbar_arrive_expect_tx(smem_u32(&xfull[s]), stage_x);
                     for (int r = 0; r < p.BN; r += kXBoxRows)
                         tma_load_2d(X_of(s) + static_cast<uint32_t>(r) * 128u, &tm_x, kb * kBK, m0 + r,
                                     smem_u32(&xfull[s]), pol);
                 }
             }
+            // every issued copy has landed before the CTA may exit
+            for (int u = it > SX ? it - SX : 0; u < it; ++u)
+                if (!mbar_wait(smem_u32(&xfull[u % SX]), (u / SX) & 1, p.status)) break;
         }
     } else if (warp == 2) {
         // ---------------- weight producer: packed codes, scales, biases ----------------
@@ -304,13 +312,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol = policy_evict_last();  // each weight tile serves every activation tile
             bool ok = true;
             int it = 0, sbi = 0;
-            for (int t = 0; t < my_units; ++t) {
+            for (int t = 0; t < my_units && ok; ++t) {
                 int tile, split, n0, m0, kb0, kb1;
                 unit_of(t, tile, split, n0, m0, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     if (p.sb_tma && (kb == kb0 || kb % p.sg == 0)) {  // the scale/bias box holding kb
                         const int ss = sbi % kSSB;
-                        if (sbi >= kSSB && ok) ok = mbar_wait(smem_u32(&sbempty[ss]), ((sbi / kSSB) - 1) & 1, p.status);
+                        if (sbi >= kSSB) ok = mbar_wait(smem_u32(&sbempty[ss]), ((sbi / kSSB) - 1) & 1, p.status);
+                        if (!ok) break;  // the slot may still be in use: issue nothing more
                         mbar_arrive_expect_tx(smem_u32(&sbfull[ss]), 2u * kStageSB);
                         const int g0 = (kb / p.sg) * kSbGroups;
                         tma_load_2d(SC_of(ss), &tm_scales, g0, n0, smem_u32(&sbfull[ss]), pol);
@@ -318,28 +327,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ++sbi;
                     }
                     const int sp = it % kSP;
-                    if (it >= kSP && ok) ok = mbar_wait(smem_u32(&pempty[sp]), ((it / kSP) - 1) & 1, p.status);
+                    if (it >= kSP) ok = mbar_wait(smem_u32(&pempty[sp]), ((it / kSP) - 1) & 1, p.status);
+                    if (!ok) break;
                     mbar_arrive_expect_tx(smem_u32(&pfull[sp]), kStageP);
                     tma_load_2d(P_of(sp), &tm_packed, kb * kBK, n0, smem_u32(&pfull[sp]), pol);
                 }
             }
+            // every issued copy has landed before the CTA may exit (on a
+            // break above, `it` counts the code loads actually issued)
+            for (int u = it > kSP ? it - kSP : 0; u < it; ++u)
+                if (!mbar_wait(smem_u32(&pfull[u % kSP]), (u / kSP) & 1, p.status)) break;
+            for (int u = sbi > kSSB ? sbi - kSSB : 0; u < sbi; ++u)
+                if (!mbar_wait(smem_u32(&sbfull[u % kSSB]), (u / kSSB) & 1, p.status)) break;
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             bool ok = true;
             int it = 0;
-            for (int t = 0; t < my_units; ++t) {
+            for (int t = 0; t < my_units && ok; ++t) {
                 int tile, split, n0, m0, kb0, kb1;
                 unit_of(t, tile, split, n0, m0, kb0, kb1);
                 // the epilogue must have drained the accumulators (previous unit)
-                if (t >= 1 && ok) ok = mbar_wait(smem_u32(acc_empty), (t - 1) & 1, p.status);
+                if (t >= 1) ok = mbar_wait(smem_u32(acc_empty), (t - 1) & 1, p.status);
+                if (!ok) break;  // issue no MMA into accumulators still being read
                 tc_fence_after();
                 const uint32_t d0 = tmem_base, d1 = tmem_base + p.tmem_cols;
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S, sx = it % SX;
-                    if (ok) ok = mbar_wait(smem_u32(&full[s]), (it / S) & 1, p.status);
+                    ok = mbar_wait(smem_u32(&full[s]), (it / S) & 1, p.status);
                     if (ok) ok = mbar_wait(smem_u32(&xfull[sx]), (it / SX) & 1, p.status);
+                    if (!ok) break;  // operands not there: issue nothing more
                     tc_fence_after();
                     const uint64_t a0 = sw128_kmajor_desc(A_of(s));
                     const uint64_t a1 = sw128_kmajor_desc(A_of(s) + kHM * 128u);
@@ -354,8 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_commit(smem_u32(&empty[s]));
                     umma_commit(smem_u32(&xempty[sx]));
                 }
-                umma_commit(smem_u32(acc_full));
+                if (ok) umma_commit(smem_u32(acc_full));
             }
+            // every MMA this thread issued has finished before TMEM is freed
+            umma_commit(smem_u32(drain));
+            mbar_wait(smem_u32(drain), 0, p.status);
         }
         __syncwarp();
     } else if (warp < kFirstEpilogue) {

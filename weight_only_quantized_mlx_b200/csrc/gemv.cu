@@ -396,6 +396,7 @@ GemvParams base_params(const WeightView& w, const StreamPlan& pl) {
 cudaError_t launch_gemv(const WeightView& w, int mode, const void* x, const void* gate,
                         const void* up, const void* resid, void* y, cudaStream_t stream) {
     if (w.N == 0) return cudaSuccess;
+    if (gemv_la_supported(w, mode, x, gate, up)) return launch_gemv_la(w, mode, x, gate, up, resid, y, stream);
     if (stream_mma_supported(w, mode, 1, x, gate, up))
         return launch_stream_mma(w, mode, 1, x, gate, up, resid, y, stream);
     const bool acts_aligned = (mode == GEMV_PLAIN) ? a16(x) : (a16(gate) && a16(up));

@@ -147,9 +147,11 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
             const uint64_t pol = policy_evict_first();
             [[maybe_unused]] const uint64_t pol_x = XS ? policy_evict_last() : 0ull;  // every CTA reads the same activations
             bool ok = true;
+            int issued = 0;
             for (int kb = 0; kb < p.num_kb; ++kb) {
                 const int s = kb % S;
-                if (kb >= S && ok) ok = mbar_wait(smem_u32(&empty[s]), ((kb / S) - 1) & 1, p.status);
+                if (kb >= S) ok = mbar_wait(smem_u32(&empty[s]), ((kb / S) - 1) & 1, p.status);
+                if (!ok) break;  // consumers may still be reading this slot: issue nothing more
                 const int col0 = kb * kKB;
                 int nbox = (p.K - col0 + 127) / 128;
                 if (nbox > NB) nbox = NB;
@@ -165,7 +167,11 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
                     for (int j = 0; j < kKB / 64; ++j)
                         tma_load_2d(st + p.x_off + static_cast<uint32_t>(j) * p.xbox_bytes, tm_x, col0 + 64 * j, 0, bar,
                                     pol_x);
+                issued = kb + 1;
             }
+            // every issued copy has landed before the CTA may exit
+            for (int kb = issued > S ? issued - S : 0; kb < issued; ++kb)
+                if (!mbar_wait(smem_u32(&full[kb % S]), (kb / S) & 1, p.status)) break;
         }
         return;
     }

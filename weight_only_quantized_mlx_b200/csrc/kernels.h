@@ -27,6 +27,7 @@ struct DeviceInfo {
     int device;
     int sm_count;
     int max_smem_optin;
+    int smem_per_sm;  // shared memory of one SM (bytes), for co-resident CTAs
 };
 const DeviceInfo& device_info();
 
@@ -78,6 +79,12 @@ cudaError_t launch_dequant_as(const WeightView& w, void* out, int dtype, cudaStr
 // mlx_int8_gemv family (m = 1): y = W h (+ resid), h = x or silu(gate)*up.
 cudaError_t launch_gemv(const WeightView& w, int mode, const void* x, const void* gate,
                         const void* up, const void* resid, void* y, cudaStream_t stream);
+
+// m = 1 stream kernel (gemv and its silu variants) with fixed per-warp work
+// items; N up to 128 rows per SM.
+bool gemv_la_supported(const WeightView& w, int mode, const void* x, const void* gate, const void* up);
+cudaError_t launch_gemv_la(const WeightView& w, int mode, const void* x, const void* gate, const void* up,
+                           const void* resid, void* y, cudaStream_t stream);
 
 // Tensor-pipe stream kernel (mma.sync fragments) for m <= kStreamMmaMaxM:
 // gemv and its silu variants (m == 1) and small-m gemm (plain mode).
