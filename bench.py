@@ -195,8 +195,10 @@ def time_region(fn, steps, warmup, stream, world):
     return max_over_ranks(ms, world, device="cuda")
 
 
-def upload_weight(mq, p, s, b, gs):
-    return mq.MlxInt8Weight.load(__import__("synth").weight_blob("w", p, s, b), "w", gs)
+def upload_weight(mq, p, s, b, gs, static=True):
+    """Load a synthetic weight.  Benchmark weights are loaded once and only
+    read, so they carry MLXQ_WEIGHT_STATIC unless static=False."""
+    return mq.MlxInt8Weight.load(__import__("synth").weight_blob("w", p, s, b), "w", gs, static=static)
 
 
 def run_gpu(args):
@@ -249,6 +251,19 @@ def run_gpu(args):
     with ClockSampler(dev.index or 0) as clk:
         ms = time_region(graph.replay, args.steps, args.warmup, stream, world)
         ms_eager = time_region(lambda: step_on(s_ptr), args.steps, args.warmup, stream, world)
+        # the same graph with the weights' flags cleared: every weight read
+        # then waits for the previous launch
+        for w in weights:
+            w.handle.flags = 0
+        step_on(s_ptr)
+        torch.cuda.synchronize()
+        graph_plain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_plain):
+            step_on(torch.cuda.current_stream().cuda_stream)
+        ms_plain = time_region(graph_plain.replay, args.steps, args.warmup, stream, world)
+        del graph_plain
+        for w in weights:
+            w.handle.flags = mq.MLXQ_WEIGHT_STATIC
         # e2e: the public call with host buffers.  Every step copies its 100
         # activation vectors from pinned host memory in one H2D, makes the 100
         # mlxq_gemv calls, and reads the 100 results back in one D2H, all
@@ -278,7 +293,7 @@ def run_gpu(args):
     e2e_value = total_bytes / (ms_e2e * 1e-3) / 1e9
     achieved = per_launch / (ms * 1e-3 / N_PAIRS) / 1e9
     traffic = profile_traffic("gemv_decode_4096x4096_gs64", [
-        "weight_only_quantized_mlx_b200/csrc/gemv_mma.cu",
+        "weight_only_quantized_mlx_b200/csrc/gemv_la.cu",
         "weight_only_quantized_mlx_b200/csrc/device_common.cuh"])
     out = {
         "metric": "W8 group-affine GEMV HBM GB/s (% of peak) at m=1; gemm TFLOP/s at m=4096",
@@ -301,12 +316,14 @@ def run_gpu(args):
             "weights": "u8 group-affine, bf16 scale/bias", "activations": "bf16",
             "accumulate": "fp32", "parallelism": f"dp{world} (independent problems)",
             "launch": "CUDA graph of the step's 100 launches",
+            "weight_flags": "MLXQ_WEIGHT_STATIC (weights loaded once, never written)",
             "eager_gbs": round(total_bytes / (ms_eager * 1e-3) / 1e9, 1),
+            "graph_gbs_without_static_flag": round(total_bytes / (ms_plain * 1e-3) / 1e9, 1),
         },
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-            "peak_source": peaks["source"], "kernel": "k_stream_mma (mlx_int8_gemv)",
+            "peak_source": peaks["source"], "kernel": "k_gemv_la (mlx_int8_gemv)",
         },
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": 2 * D_K * N_PAIRS, "d2h_bytes_per_step": 2 * D_N * N_PAIRS},
@@ -351,7 +368,7 @@ def measure_rows(mq, torch, synth, dev, stream, dec_weights, peaks, args):
 
     # quantize: BF16 [4096, 4096] -> codes + tables, 8 sources rotating (268 MB)
     qsrc = [torch.randn(D_N, D_K, device=dev).to(torch.bfloat16) * 0.04 for _ in range(8)]
-    qdst = upload_weight(mq, *synth.weight(synth.rng(5000), D_N, D_K, D_GS), D_GS)
+    qdst = upload_weight(mq, *synth.weight(synth.rng(5000), D_N, D_K, D_GS), D_GS, static=False)
     qturn = [0]
 
     def quant():
@@ -537,7 +554,7 @@ def run_reference(args):
 def run_case(args):
     """--case KIND:N:K:GS[:M]: run one kernel `--steps` times on a seeded
     weight, no timing line (the command the committed ncu summaries use).
-    KIND is dequant, gemv, silu, resid, gemm (auto), smallm, rows or tc."""
+    KIND is dequant, quantize, gemv, silu, resid, gemm (auto), smallm, rows or tc."""
     import torch
     import synth
     import weight_only_quantized_mlx_b200 as mq
@@ -554,11 +571,17 @@ def run_case(args):
     r = to_dev(synth.activations(g, N))
     Y = torch.empty(m, N, dtype=torch.bfloat16, device=dev)
     out = torch.empty(N * K, dtype=torch.bfloat16, device=dev) if kind == "dequant" else None
+    wsrc = to_dev(synth.activations(g, N, K)) if kind == "quantize" else None
+    if kind == "quantize":
+        w.release()
+        w = upload_weight(mq, *synth.weight(g, N, K, gs), gs, static=False)  # the destination is written
     kernel = {"gemm": mq.MLXQ_GEMM_AUTO, "smallm": mq.MLXQ_GEMM_SMALLM, "rows": mq.MLXQ_GEMM_ROWS,
               "tc": mq.MLXQ_GEMM_TCGEN05}.get(kind)
     for _ in range(args.steps):
         if kind == "dequant":
             mq.mlxq_dequant(w.handle, out)
+        elif kind == "quantize":
+            mq.mlxq_quantize(wsrc, w.handle)
         elif kind == "gemv":
             mq.mlxq_gemv(w.handle, X, Y)
         elif kind == "silu":

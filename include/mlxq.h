@@ -66,7 +66,8 @@ enum {
  * A handle filled by mlxq_load owns its three buffers and must be freed once
  * with mlxq_release.  A caller may instead fill the struct with device
  * buffers it owns (same layouts); such a handle must not be passed to
- * mlxq_release.
+ * mlxq_release.  `flags` is 0 or a combination of MLXQ_WEIGHT_* below;
+ * mlxq_load sets it to 0 and a caller may change it afterwards.
  */
 typedef struct mlxq_weight {
     void* packed;          /* uint32 [N, K/4] */
@@ -75,7 +76,19 @@ typedef struct mlxq_weight {
     uint32_t out_features; /* N */
     uint32_t in_features;  /* K (a multiple of 4) */
     uint32_t group_size;   /* gs, divides K */
+    uint32_t flags;        /* MLXQ_WEIGHT_* */
 } mlxq_weight;
+
+/*
+ * MLXQ_WEIGHT_STATIC: the caller guarantees that while a call that reads this
+ * weight is queued or running, no kernel on any stream writes its packed,
+ * scales or biases buffers (true of weights loaded once and then only read,
+ * as in decoding).  The m = 1 kernels may then copy the weight into shared
+ * memory before the previous work on the stream has finished; activations,
+ * residuals and outputs are still touched only after it.  Off (0) by default:
+ * every read of the weight then comes after the previous work on the stream.
+ */
+#define MLXQ_WEIGHT_STATIC 1u
 
 /*
  * mlxq_load (page: MlxInt8Weight::load).  Parses an in-memory safetensors

@@ -180,6 +180,24 @@ def _fake_weight(N=8, K=64, gs=32):
     return mq.mlxq_weight(0x10000, 0x20000, 0x30000, N, K, gs)
 
 
+def test_unknown_weight_flags_are_refused():
+    L = mq.lib()
+    w = _fake_weight()
+    w.flags = 0x2  # not a defined MLXQ_WEIGHT_* bit
+    X, Y = 0x100000, 0x200000
+    assert L.mlxq_gemv(ctypes.byref(w), X, Y, 0) == mq.MLXQ_ERR_INVALID_ARG
+    assert "flags" in mq.mlxq_last_error()
+    assert L.mlxq_dequant(ctypes.byref(w), Y, 0) == mq.MLXQ_ERR_INVALID_ARG
+
+
+def test_weight_struct_layout_has_flags_last():
+    # the C struct: three pointers, three uint32 dimensions, uint32 flags
+    assert [f[0] for f in mq.mlxq_weight._fields_] == ["packed", "scales", "biases", "out_features",
+                                                      "in_features", "group_size", "flags"]
+    assert ctypes.sizeof(mq.mlxq_weight) == 3 * 8 + 4 * 4
+    assert mq.MLXQ_WEIGHT_STATIC == 1
+
+
 def test_release_twice_is_refused():
     w = mq.mlxq_weight()
     assert mq.lib().mlxq_release(ctypes.byref(w)) == mq.MLXQ_ERR_INVALID_ARG

@@ -335,6 +335,75 @@ def test_quantize_then_gemv():
     assert_close(host_bits(y), oracle.gemv(*host, gs, x), "gemv of a quantised weight")
 
 
+def test_gemv_reads_a_weight_written_just_before():
+    # Without MLXQ_WEIGHT_STATIC every read of the weight follows the previous
+    # work on the stream: a gemv queued right behind the quantize that writes
+    # its weight (no synchronisation in between) sees the new codes, round
+    # after round.
+    g = synth.rng(62)
+    N, K, gs = 4096, 4096, 64
+    dst_t = (torch.zeros(N, K // 4, dtype=torch.int32, device="cuda"),
+             torch.zeros(N, K // gs, dtype=torch.int16, device="cuda"),
+             torch.zeros(N, K // gs, dtype=torch.int16, device="cuda"))
+    dst = mq.weight_view(*dst_t, gs)
+    x = synth.activations(g, K)
+    xd = dev(x)
+    ws = [synth.to_bf16_bits((g.standard_normal((N, K)) * s).astype(np.float32)) for s in (0.05, 0.02, 0.08)]
+    wd = [dev(w) for w in ws]
+    ys = [torch.empty(N, dtype=torch.bfloat16, device="cuda") for _ in ws]
+    torch.cuda.synchronize()
+    for wi, yi in zip(wd, ys):
+        mq.mlxq_quantize(wi, dst)
+        mq.mlxq_gemv(dst, xd, yi)
+    torch.cuda.synchronize()
+    for w, yi in zip(ws, ys):
+        assert_close(host_bits(yi), oracle.gemv(*oracle.quantize(w, gs), gs, x), "gemv right after quantize")
+
+
+@pytest.mark.parametrize("N,K,gs", [(4096, 4096, 64), (4096, 14336, 64), (1000, 4096, 128), (333, 1024, 32)])
+def test_static_weight_flag(N, K, gs):
+    # MLXQ_WEIGHT_STATIC lets the weight's copies start before the previous
+    # work has finished; the results are identical to the default
+    W, g = make(63, N, K, gs)
+    x = synth.activations(g, K)
+    gate, up, r = synth.activations(g, K), synth.activations(g, K), synth.activations(g, N)
+    Ws = DevWeight(*W.host, gs)
+    Ws.w.flags = mq.MLXQ_WEIGHT_STATIC
+    y0, y1 = run_gemv(W, x), run_gemv(Ws, x)
+    assert np.array_equal(y0, y1)
+    assert_close(y1, oracle.gemv(*W.host, gs, x), f"static gemv {N}x{K}")
+    outs = []
+    for Wx in (W, Ws):
+        y = Guarded(N)
+        mq.mlxq_gemv_silu_gate_resid(Wx.w, dev(gate), dev(up), dev(r), y.data_ptr())
+        torch.cuda.synchronize()
+        y.check_guards()
+        outs.append(y.value_bits())
+    assert np.array_equal(outs[0], outs[1])
+    assert_close(outs[1], oracle.silu_gate_resid(*W.host, gs, gate, up, r), f"static resid {N}x{K}")
+
+
+def test_static_weight_decode_chain():
+    # a chain of static-weight gemvs, each reading the previous one's output,
+    # with no synchronisation: the activations are still read after they are
+    # written
+    g = synth.rng(64)
+    N = K = 4096
+    Ws = []
+    for _ in range(6):
+        W, _ = make(int(g.integers(1 << 30)), N, K, 64)
+        W.w.flags = mq.MLXQ_WEIGHT_STATIC
+        Ws.append(W)
+    x = synth.activations(g, K)
+    bufs = [dev(x)] + [torch.empty(N, dtype=torch.bfloat16, device="cuda") for _ in Ws]
+    for i, W in enumerate(Ws):
+        mq.mlxq_gemv(W.w, bufs[i], bufs[i + 1])
+    torch.cuda.synchronize()
+    for i, W in enumerate(Ws):
+        xin = host_bits(bufs[i])
+        assert_close(host_bits(bufs[i + 1]), oracle.gemv(*W.host, 64, xin), f"chain step {i}")
+
+
 def test_quantize_constant_and_signed_zero_groups():
     # range 0 (scale 0, codes 0) and groups of signed zeros: the first
     # minimum in column order decides the bias's sign, as in the oracle
@@ -359,7 +428,8 @@ def run_gemm(W, X_bits, m, kernel=mq.MLXQ_GEMM_AUTO):
     return Y.value_bits().reshape(m, W.N)
 
 
-SMALLM_SHAPES = [(512, 1024, 64), (300, 4096, 32), (256, 14336, 128), (128, 28672, 64), (77, 512, 16)]
+SMALLM_SHAPES = [(512, 1024, 64), (300, 4096, 32), (256, 14336, 128), (128, 28672, 64), (77, 512, 16),
+                 (5000, 1152, 16), (2100, 2304, 32)]   # several tile groups per CTA; K not a multiple of 512
 
 
 @pytest.mark.parametrize("N,K,gs", SMALLM_SHAPES)

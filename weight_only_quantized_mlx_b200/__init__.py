@@ -36,6 +36,8 @@ MLXQ_GEMM_SMALLM = 2
 MLXQ_GEMM_TCGEN05 = 3
 MLXQ_GEMM_SMALLM_FFMA = 4
 
+MLXQ_WEIGHT_STATIC = 1
+
 MLXQ_DTYPE_BF16 = 0
 MLXQ_DTYPE_F16 = 1
 MLXQ_DTYPE_F32 = 2
@@ -50,7 +52,8 @@ class mlxq_weight(ctypes.Structure):
     """C ``mlxq_weight``: three device pointers and the dimensions."""
     _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("biases", ctypes.c_void_p), ("out_features", ctypes.c_uint32),
-                ("in_features", ctypes.c_uint32), ("group_size", ctypes.c_uint32)]
+                ("in_features", ctypes.c_uint32), ("group_size", ctypes.c_uint32),
+                ("flags", ctypes.c_uint32)]
 
 
 class MlxqError(RuntimeError):
@@ -183,12 +186,12 @@ def mlxq_selftest_fail_alloc(nth: int) -> None:
     _check(lib().mlxq_selftest_fail_alloc(nth))
 
 
-def weight_view(packed, scales, biases, group_size: int) -> mlxq_weight:
+def weight_view(packed, scales, biases, group_size: int, flags: int = 0) -> mlxq_weight:
     """A non-owning handle over caller-owned device tensors (packed uint32/int32
     [N, K/4], scales/biases bf16 [N, K/gs]).  Never pass it to mlxq_release."""
     N = packed.shape[0]
     K = packed.shape[1] * 4
-    return mlxq_weight(_ptr(packed), _ptr(scales), _ptr(biases), N, K, group_size)
+    return mlxq_weight(_ptr(packed), _ptr(scales), _ptr(biases), N, K, group_size, flags)
 
 
 class MlxInt8Weight:
@@ -201,8 +204,13 @@ class MlxInt8Weight:
         self.owned = owned
 
     @classmethod
-    def load(cls, blob: bytes, base: str, group_size: int) -> "MlxInt8Weight":
-        return cls(mlxq_load(blob, base, group_size), True)
+    def load(cls, blob: bytes, base: str, group_size: int, static: bool = False) -> "MlxInt8Weight":
+        """static=True sets MLXQ_WEIGHT_STATIC (see include/mlxq.h): the caller
+        promises that no kernel writes the weight while calls read it."""
+        w = cls(mlxq_load(blob, base, group_size), True)
+        if static:
+            w.handle.flags |= MLXQ_WEIGHT_STATIC
+        return w
 
     @property
     def out_features(self) -> int:

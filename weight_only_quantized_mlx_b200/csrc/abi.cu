@@ -351,6 +351,9 @@ int check_weight(const mlxq_weight* w, WeightView& v) {
     v.K = w->in_features;
     v.gs = w->group_size;
     v.G = v.K / v.gs;
+    if (w->flags & ~MLXQ_WEIGHT_STATIC)
+        return fail(MLXQ_ERR_INVALID_ARG, "unknown weight flags 0x%x", w->flags & ~MLXQ_WEIGHT_STATIC);
+    v.flags = w->flags;
     return MLXQ_OK;
 }
 
@@ -509,6 +512,7 @@ int mlxq_load(const void* blob, size_t blob_len, const char* base, uint32_t grou
     out->out_features = static_cast<uint32_t>(N);
     out->in_features = static_cast<uint32_t>(K);
     out->group_size = group_size;
+    out->flags = 0;
     return ok();
 }
 
@@ -610,7 +614,8 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
     int k = kernel;
     if (k == MLXQ_GEMM_AUTO) {
         if (M == 1) k = MLXQ_GEMM_ROWS;
-        else if (M <= kStreamMmaMaxM && stream_mma_supported(v, GEMV_PLAIN, M, x, nullptr, nullptr)) k = MLXQ_GEMM_SMALLM;
+        else if (M <= kStreamMmaMaxM && stream_mma_supported(v, GEMV_PLAIN, M, x, nullptr, nullptr))
+            k = MLXQ_GEMM_SMALLM;
         else if (gemm_tc_supported(v, M, x, y)) k = MLXQ_GEMM_TCGEN05;
         else if (M <= kSmallMMax && x16 && gemm_smallm_supported(v, M)) k = MLXQ_GEMM_SMALLM_FFMA;
         else k = MLXQ_GEMM_ROWS;

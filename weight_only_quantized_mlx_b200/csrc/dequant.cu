@@ -1,8 +1,8 @@
 // mlx_int8_dequant ("MlxInt8Weight" page, dequantize_to): write the full
 // weight as BF16, out[n, k] = bf16_rne(fma_f32(scale[n,g], q[n,k], bias[n,g])).
 //
-// HBM-bound streaming kernel: each thread turns 16-byte word groups (16
-// codes each) into pairs of 16-byte BF16 stores.  s*q is exact in fp32, so the only
+// HBM-bound streaming kernel: each thread turns one 16-byte word group (16
+// codes) into two 16-byte BF16 stores.  s*q is exact in fp32, so the only
 // roundings are the fp32 add inside the fma and the final RNE to BF16; the
 // result is bit-identical to any correct fp32 implementation of the formula.
 #include <cuda_fp16.h>
@@ -16,56 +16,37 @@ namespace mlxq {
 namespace {
 
 // Fast path: K % 16 == 0, group_size % 16 == 0, 16-byte aligned buffers.
-// A thread turns kChunks 16-code chunks (16 codes never straddle a group)
-// into BF16: all its loads are issued before the first conversion, so each
-// SM keeps enough bytes in flight to cover HBM latency.  Chunk j of a pass is
-// blockDim.x chunks after chunk j - 1, so a warp's loads and stores stay
-// contiguous.
-constexpr int kChunks = 4;
-
-__global__ void __launch_bounds__(256, 4) k_dequant_vec16(const uint4* __restrict__ packed,
+// One thread per 16-code chunk; a chunk never straddles a group.
+__global__ void __launch_bounds__(256) k_dequant_vec16(const uint4* __restrict__ packed,
                                                        const uint16_t* __restrict__ scales,
                                                        const uint16_t* __restrict__ biases,
                                                        uint4* __restrict__ out, int64_t nchunks,
                                                        int64_t chunks_per_row,
                                                        int64_t chunks_per_group, int64_t G) {
-    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x * kChunks;
-    for (int64_t c0 = static_cast<int64_t>(blockIdx.x) * blockDim.x * kChunks + threadIdx.x; c0 < nchunks;
-         c0 += step) {
-        uint4 wq[kChunks];
-        float s[kChunks], b[kChunks];
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < nchunks;
+         c += stride) {
+        const int64_t n = c / chunks_per_row;
+        const int64_t j = c - n * chunks_per_row;
+        const int64_t gi = n * G + j / chunks_per_group;
+        const uint4 wq = ldg_nc_v4(packed + c);
+        const float s = bf16_bits_to_f32(__ldg(scales + gi));
+        const float b = bf16_bits_to_f32(__ldg(biases + gi));
+        const uint32_t words[4] = {wq.x, wq.y, wq.z, wq.w};
+        uint32_t o[8];
 #pragma unroll
-        for (int j = 0; j < kChunks; ++j) {
-            const int64_t c = c0 + static_cast<int64_t>(j) * blockDim.x;
-            if (c < nchunks) {
-                const int64_t n = c / chunks_per_row;
-                const int64_t gi = n * G + (c - n * chunks_per_row) / chunks_per_group;
-                wq[j] = ldg_nc_v4(packed + c);
-                s[j] = bf16_bits_to_f32(__ldg(scales + gi));
-                b[j] = bf16_bits_to_f32(__ldg(biases + gi));
-            }
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t w = words[i];
+            const float q0 = code_magic<0>(w) - kMagic;
+            const float q1 = code_magic<1>(w) - kMagic;
+            const float q2 = code_magic<2>(w) - kMagic;
+            const float q3 = code_magic<3>(w) - kMagic;
+            o[2 * i] = pack_bf16x2(__fmaf_rn(s, q0, b), __fmaf_rn(s, q1, b));
+            o[2 * i + 1] = pack_bf16x2(__fmaf_rn(s, q2, b), __fmaf_rn(s, q3, b));
         }
-#pragma unroll
-        for (int j = 0; j < kChunks; ++j) {
-            const int64_t c = c0 + static_cast<int64_t>(j) * blockDim.x;
-            if (c < nchunks) {
-                const uint32_t words[4] = {wq[j].x, wq[j].y, wq[j].z, wq[j].w};
-                uint32_t o[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w = words[i];
-                    const float q0 = code_magic<0>(w) - kMagic;
-                    const float q1 = code_magic<1>(w) - kMagic;
-                    const float q2 = code_magic<2>(w) - kMagic;
-                    const float q3 = code_magic<3>(w) - kMagic;
-                    o[2 * i] = pack_bf16x2(__fmaf_rn(s[j], q0, b[j]), __fmaf_rn(s[j], q1, b[j]));
-                    o[2 * i + 1] = pack_bf16x2(__fmaf_rn(s[j], q2, b[j]), __fmaf_rn(s[j], q3, b[j]));
-                }
-                uint4* dst = out + 2 * c;
-                __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
-                __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
-            }
-        }
+        uint4* dst = out + 2 * c;
+        __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+        __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
     }
 }
 
@@ -153,8 +134,8 @@ cudaError_t launch_dequant(const WeightView& w, void* out, cudaStream_t stream) 
                      aligned16(out);
     if (vec) {
         const int64_t nchunks = total / 16;
-        int64_t blocks = (nchunks + 256 * kChunks - 1) / (256 * kChunks);
-        const int64_t cap = static_cast<int64_t>(sms) * 4;  // 4 resident blocks of 256 per SM: one wave
+        int64_t blocks = (nchunks + 255) / 256;
+        const int64_t cap = static_cast<int64_t>(sms) * 32;
         if (blocks > cap) blocks = cap;
         k_dequant_vec16<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
             reinterpret_cast<const uint4*>(w.packed), w.scales, w.biases,

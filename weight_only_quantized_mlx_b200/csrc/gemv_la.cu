@@ -30,7 +30,7 @@ namespace {
 
 constexpr int kLaMaxPairs = 8;   // 16-row tiles per CTA (R <= 128)
 constexpr int kLaMaxStages = 8;
-constexpr int kLaSlices = 8;     // 64 * CPL-code slices of a stage
+constexpr int kLaSlices = 8;     // 64 * CPL-code slices of a stage, one per item
 
 struct LaParams {
     const uint16_t* x;
@@ -44,6 +44,7 @@ struct LaParams {
     int gpk;                 // scale groups per stage
     int Kpad;                // num_kb * stage width (activation staging, zero past K)
     int pf_stages;           // stages prefetched to L2 before the dependency wait
+    int pre_wait;            // stages copied into shared memory before it (static weights; <= S)
     uint32_t box_bytes;      // npair * 16 rows * 128 bytes
     uint32_t sb_bytes;       // one table (scales or biases) of a stage, 128-byte padded
     uint32_t stage_bytes;    // 1024-byte multiple
@@ -81,14 +82,14 @@ __device__ __forceinline__ float silu_fast(float t) { return __fdividef(t, 1.0f 
 // W consumer warps (+ one producer warp).  A stage's work items are
 // (16-row tile, 64 * CPL-code slice) pairs, npair * 8 of them; warp w takes
 // items w, w + W, ... (at most JMAX), the same ones in every stage, so each
-// item has its own accumulators.  CPL: 16-code chunks per lane per item (1,
-// or 2 when the group size needs 1024-code stages); GS: group size.
+// item has its own accumulators.  CPL: 16-code chunks per lane per item (1, 2
+// or 4; stages of 512 * CPL codes); GS: group size.
 template <int MODE, int CPL, int GS, int W, int JMAX>
 __global__ void __launch_bounds__((W + 1) * 32, 1)
     k_gemv_la(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_scales,
               const __grid_constant__ CUtensorMap tm_biases, const LaParams p) {
-    constexpr int kKB = 512 * CPL;   // codes per stage
-    constexpr int kNB = 4 * CPL;     // 128-code boxes per stage
+    constexpr int kKB = 64 * CPL * kLaSlices;  // codes per stage
+    constexpr int kNB = kKB / 128;      // 128-code boxes per stage
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -120,18 +121,22 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             prefetch_tmap(&tm_packed);
             prefetch_tmap(&tm_scales);
             prefetch_tmap(&tm_biases);
-            // Warm L2 with the first stages while the previous launch finishes.
+            // Warm L2 with the first stages while the previous launch finishes
+            // (when their copies must wait for it).
             for (int kb = 0; kb < p.pf_stages; ++kb) {
                 for (int b = 0; b < kNB && kb * kKB + 128 * b < p.K; ++b)
                     tma_prefetch_l2_2d(&tm_packed, kb * kKB + 128 * b, r0);
                 tma_prefetch_l2_2d(&tm_scales, kb * p.gpk, r0);
                 tma_prefetch_l2_2d(&tm_biases, kb * p.gpk, r0);
             }
-            pdl_wait();
             const uint64_t pol = policy_evict_first();
             bool ok = true;
             int issued = 0;
+            // Stages [0, pre_wait) of a weight no running kernel writes are
+            // copied before the dependency wait; everything else after it.
+            if (p.pre_wait == 0) pdl_wait();
             for (int kb = 0; kb < p.num_kb; ++kb) {
+                if (kb == p.pre_wait && kb > 0) pdl_wait();
                 const int s = kb % S;
                 if (kb >= S) ok = mbar_wait(smem_u32(&empty[s]), ((kb / S) - 1) & 1, p.status);
                 if (!ok) break;  // stop issuing: consumers may still be reading this slot
@@ -148,6 +153,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                 tma_load_2d(st + kNB * p.box_bytes + p.sb_bytes, &tm_biases, kb * p.gpk, r0, bar, pol);
                 issued = kb + 1;
             }
+            if (p.pre_wait >= p.num_kb) pdl_wait();
             // Leave only once every issued copy has landed (bounded; normally
             // the consumers have already waited for all of them).
             for (int kb = issued > S ? issued - S : 0; kb < issued; ++kb)
@@ -216,33 +222,55 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         for (int j = 0; j < JMAX; ++j) {
             const int it = warp + W * j;
             if (it < items) {  // warp-uniform
-                const int pj = it >> 3, sl = it & 7;
-                const int b = CPL == 1 ? (sl >> 1) : sl;
+                const int pj = it / kLaSlices, sl = it % kLaSlices;
                 const uint32_t row = static_cast<uint32_t>(16 * pj + g);
-                const uint32_t boxa = st + static_cast<uint32_t>(b) * p.box_bytes + row * 128u;
+                // An item is CPL / 2 boxes (one half box when CPL == 1); per box
+                // the lane takes chunks 2 tq and 2 tq + 1 (CPL >= 2) or the
+                // slice's one (CPL == 1), which share a scale group when the
+                // group spans 32 codes or more.
 #pragma unroll
-                for (int ci = 0; ci < CPL; ++ci) {
-                    const int c = 2 * tq + (CPL == 1 ? (sl & 1) : ci);
-                    const int kc = kb * kKB + 128 * b + 16 * c;
-                    const uint4 x0 = lds128(xrow + 2u * kc), x1 = lds128(xrow + 2u * kc + 16u);
-                    const uint32_t swz = static_cast<uint32_t>(c ^ g) << 4;
-                    const uint4 wu = lds128(boxa + swz);
-                    const uint4 wv = lds128(boxa + 8u * 128u + swz);
-                    const uint32_t so = (row * p.gpk + static_cast<uint32_t>((128 * b + 16 * c) / GS)) * 2u;
-                    const float2 s2 = make_float2(bf16_bits_to_f32(lds16(sca + so)), bf16_bits_to_f32(lds16(sca + so + sb8)));
-                    const float2 b2 = make_float2(bf16_bits_to_f32(lds16(bia + so)), bf16_bits_to_f32(lds16(bia + so + sb8)));
-                    const uint32_t uu[4] = {wu.x, wu.y, wu.z, wu.w}, vv[4] = {wv.x, wv.y, wv.z, wv.w};
-                    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                for (int hb = 0; hb < (CPL + 1) / 2; ++hb) {
+                    constexpr int kC = CPL == 1 ? 1 : 2;  // chunks of this box
+                    constexpr bool kOneGroup = kC == 1 || GS >= 32;
+                    const int b = CPL == 1 ? (sl >> 1) : sl * (CPL / 2) + hb;
+                    const uint32_t boxa = st + static_cast<uint32_t>(b) * p.box_bytes + row * 128u;
+                    // operands, shared memory -> registers
+                    uint4 xa[kC], xb[kC], wu[kC], wv[kC];
+                    float2 s2[kOneGroup ? 1 : kC], b2[kOneGroup ? 1 : kC];
 #pragma unroll
-                    for (int w4 = 0; w4 < 4; ++w4) {
-                        uint32_t a0, a1, a2, a3;
-                        dequant_rows(uu[w4], vv[w4], s2, b2, a0, a1, a2, a3);
-                        // two accumulators, so consecutive MMAs do not wait on each other
-                        mma_bf16_16816(acc[j][w4 & 1], a0, a1, a2, a3, xw[2 * w4], xw[2 * w4 + 1]);
+                    for (int ci = 0; ci < kC; ++ci) {
+                        const int c = 2 * tq + (CPL == 1 ? (sl & 1) : ci);
+                        const uint32_t xa_addr = xrow + 2u * static_cast<uint32_t>(kb * kKB + 128 * b + 16 * c);
+                        xa[ci] = lds128(xa_addr);
+                        xb[ci] = lds128(xa_addr + 16u);
+                        const uint32_t swz = static_cast<uint32_t>(c ^ g) << 4;
+                        wu[ci] = lds128(boxa + swz);
+                        wv[ci] = lds128(boxa + 8u * 128u + swz);
+                        if (!kOneGroup || ci == 0) {
+                            const uint32_t so = (row * p.gpk + static_cast<uint32_t>((128 * b + 16 * c) / GS)) * 2u;
+                            s2[ci] = make_float2(bf16_bits_to_f32(lds16(sca + so)), bf16_bits_to_f32(lds16(sca + so + sb8)));
+                            b2[ci] = make_float2(bf16_bits_to_f32(lds16(bia + so)), bf16_bits_to_f32(lds16(bia + so + sb8)));
+                        }
+                    }
+#pragma unroll
+                    for (int ci = 0; ci < kC; ++ci) {
+                        const uint32_t uu[4] = {wu[ci].x, wu[ci].y, wu[ci].z, wu[ci].w};
+                        const uint32_t vv[4] = {wv[ci].x, wv[ci].y, wv[ci].z, wv[ci].w};
+                        const uint32_t xw[8] = {xa[ci].x, xa[ci].y, xa[ci].z, xa[ci].w, xb[ci].x, xb[ci].y, xb[ci].z, xb[ci].w};
+                        const int gi = kOneGroup ? 0 : ci;
+#pragma unroll
+                        for (int w4 = 0; w4 < 4; ++w4) {
+                            uint32_t a0, a1, a2, a3;
+                            dequant_rows(uu[w4], vv[w4], s2[gi], b2[gi], a0, a1, a2, a3);
+                            // two accumulators, so consecutive MMAs do not wait on each other
+                            mma_bf16_16816(acc[j][w4 & 1], a0, a1, a2, a3, xw[2 * w4], xw[2 * w4 + 1]);
+                        }
                     }
                 }
             }
         }
+        // release the slot only after computing: an arrive right after the
+        // loads would make the warp wait for them before any arithmetic
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
     }
@@ -254,7 +282,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         for (int j = 0; j < JMAX; ++j) {
             const int it = warp + W * j;
             if (it < items) {
-                const int pj = it >> 3, sl = it & 7;
+                const int pj = it / kLaSlices, sl = it % kLaSlices;
                 // D columns 0 (and 1: the low part of h) of rows g and g + 8
                 const float c0 = acc[j][0][0] + acc[j][1][0], c1 = acc[j][0][1] + acc[j][1][1];
                 const float c2 = acc[j][0][2] + acc[j][1][2], c3 = acc[j][0][3] + acc[j][1][3];
@@ -275,7 +303,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     }
 }
 
-constexpr int kLaW = 16;  // consumer warps
+constexpr int kLaW = 16;        // consumer warps
+constexpr bool kLaCpl4 = false;  // 2048-code stages for short row ranges
 
 template <int MODE, int CPL, int GS, int JMAX>
 cudaError_t launch_la_t(const TensorMaps3& tm, const LaParams& p, int grid, size_t smem, cudaStream_t stream) {
@@ -288,31 +317,39 @@ cudaError_t launch_la_t(const TensorMaps3& tm, const LaParams& p, int grid, size
     return cudaGetLastError();
 }
 
+// Configurations the plan produces: CPL 4 (2048-code stages) for one or two
+// tiles, CPL 2 (1024) up to four tiles, CPL 1 (512) above, with 1, 2 or 4
+// items per warp; group size 128 always takes CPL >= 2 (16-byte table rows).
 template <int MODE, int CPL, int GS>
 cudaError_t launch_la_j(const TensorMaps3& tm, const LaParams& p, int jmax, int grid, size_t smem,
                         cudaStream_t stream) {
     if (jmax == 1) return launch_la_t<MODE, CPL, GS, 1>(tm, p, grid, smem, stream);
-    if (jmax == 2) return launch_la_t<MODE, CPL, GS, 2>(tm, p, grid, smem, stream);
-    return launch_la_t<MODE, CPL, GS, 4>(tm, p, grid, smem, stream);
+    if constexpr (CPL <= 2) {
+        if (jmax == 2) return launch_la_t<MODE, CPL, GS, 2>(tm, p, grid, smem, stream);
+        if constexpr (CPL == 1 || GS == 128) return launch_la_t<MODE, CPL, GS, 4>(tm, p, grid, smem, stream);
+    }
+    return cudaErrorInvalidValue;
 }
 
-template <int MODE, int CPL>
-cudaError_t launch_la_gs(const TensorMaps3& tm, const LaParams& p, int gs, int jmax, int grid, size_t smem,
-                         cudaStream_t stream) {
-    switch (gs) {
-        case 16: return launch_la_j<MODE, CPL, 16>(tm, p, jmax, grid, smem, stream);
-        case 32: return launch_la_j<MODE, CPL, 32>(tm, p, jmax, grid, smem, stream);
-        case 64: return launch_la_j<MODE, CPL, 64>(tm, p, jmax, grid, smem, stream);
-        default: return cudaErrorInvalidValue;
-    }
+template <int MODE, int GS>
+cudaError_t launch_la_cpl(const TensorMaps3& tm, const LaParams& p, int cpl, int jmax, int grid, size_t smem,
+                          cudaStream_t stream) {
+    if (cpl == 4) return launch_la_j<MODE, 4, GS>(tm, p, jmax, grid, smem, stream);
+    if (cpl == 2) return launch_la_j<MODE, 2, GS>(tm, p, jmax, grid, smem, stream);
+    if constexpr (GS != 128) return launch_la_j<MODE, 1, GS>(tm, p, jmax, grid, smem, stream);
+    return cudaErrorInvalidValue;
 }
 
 template <int MODE>
 cudaError_t launch_la_mode(const TensorMaps3& tm, const LaParams& p, int gs, int cpl, int jmax, int grid,
                            size_t smem, cudaStream_t stream) {
-    if (gs == 128) return launch_la_j<MODE, 2, 128>(tm, p, jmax, grid, smem, stream);
-    if (cpl == 2) return launch_la_gs<MODE, 2>(tm, p, gs, jmax, grid, smem, stream);
-    return launch_la_gs<MODE, 1>(tm, p, gs, jmax, grid, smem, stream);
+    switch (gs) {
+        case 16: return launch_la_cpl<MODE, 16>(tm, p, cpl, jmax, grid, smem, stream);
+        case 32: return launch_la_cpl<MODE, 32>(tm, p, cpl, jmax, grid, smem, stream);
+        case 64: return launch_la_cpl<MODE, 64>(tm, p, cpl, jmax, grid, smem, stream);
+        case 128: return launch_la_cpl<MODE, 128>(tm, p, cpl, jmax, grid, smem, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 bool a16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
@@ -324,37 +361,28 @@ struct LaPlan {
     size_t smem;
 };
 
-bool plan_la(const WeightView& w, int mode, LaPlan& pl) {
-    const DeviceInfo& dev = device_info();
-    if (w.N < 1 || w.K < 16 || w.K % 16 != 0 || w.K > 32768 || w.N > (1 << 30)) return false;
-    if (w.gs != 16 && w.gs != 32 && w.gs != 64 && w.gs != 128) return false;
-    if (w.G % 8 != 0) return false;  // table rows must be 16-byte multiples for the tensor copies
-    // Rows per CTA: one CTA per SM (N up to 128 rows per SM).
-    const int64_t ctas = dev.sm_count;
-    if ((w.N + ctas - 1) / ctas > kLaMaxPairs * 16) return false;
-    pl.R = static_cast<int>((w.N + ctas - 1) / ctas);
-    pl.npair = (pl.R + 15) / 16;
-    // 1024-code stages (two chunks per lane per item: half the stage
-    // synchronisations, one scale/bias load for both) while a stage of up to
-    // 4 tiles leaves room for a deep ring; wider row ranges take 512-code
-    // stages.  Group size 128 needs 1024 (a stage's tables are 16-byte rows).
-    pl.cpl = (w.gs == 128 || pl.npair <= 4) ? 2 : 1;
-    const int kb = 512 * pl.cpl;
-    pl.grid = static_cast<int>((w.N + pl.R - 1) / pl.R);
+// Stage geometry for R rows per CTA and CPL chunks per lane per item within
+// `budget` bytes of shared memory; false if not even `min_stages` stages fit.
+bool plan_geometry(const WeightView& w, int mode, int R, int cpl, size_t budget, int min_stages, LaPlan& pl) {
+    pl.R = R;
+    pl.npair = (R + 15) / 16;
+    pl.cpl = cpl;
+    const int kb = 64 * cpl * kLaSlices;
+    pl.grid = static_cast<int>((w.N + R - 1) / R);
     pl.gpk = kb / static_cast<int>(w.gs);
+    if (pl.gpk < 8) return false;  // a stage's table rows must be 16-byte multiples
     pl.num_kb = static_cast<int>((w.K + kb - 1) / kb);
     pl.Kpad = pl.num_kb * kb;
     pl.box_bytes = static_cast<uint32_t>(pl.npair) * 16u * 128u;
     pl.sb_bytes = (static_cast<uint32_t>(pl.npair) * 16u * pl.gpk * 2u + 127u) / 128u * 128u;
-    pl.stage_bytes = (4u * pl.cpl * pl.box_bytes + 2u * pl.sb_bytes + 1023u) / 1024u * 1024u;
+    pl.stage_bytes = (static_cast<uint32_t>(kb / 128) * pl.box_bytes + 2u * pl.sb_bytes + 1023u) / 1024u * 1024u;
     const uint32_t xs_bytes = static_cast<uint32_t>((mode == GEMV_PLAIN ? 2 : 4) * pl.Kpad);
     const uint32_t red_bytes = static_cast<uint32_t>(kLaSlices * pl.npair * 16 * 4);
     const size_t fixed = 1024 + xs_bytes + red_bytes + 2 * kLaMaxStages * sizeof(uint64_t);
     const int items = pl.npair * kLaSlices;
     const int j = (items + kLaW - 1) / kLaW;
     pl.jmax = j <= 1 ? 1 : (j <= 2 ? 2 : 4);
-    const size_t budget = static_cast<size_t>(dev.max_smem_optin);
-    if (budget < fixed + pl.stage_bytes) return false;
+    if (budget < fixed + static_cast<size_t>(min_stages) * pl.stage_bytes) return false;
     int S = static_cast<int>((budget - fixed) / pl.stage_bytes);
     if (S > kLaMaxStages) S = kLaMaxStages;
     if (S > pl.num_kb) S = pl.num_kb;
@@ -363,9 +391,31 @@ bool plan_la(const WeightView& w, int mode, LaPlan& pl) {
     pl.red_off = pl.xs_off + xs_bytes;
     pl.bar_off = (pl.red_off + red_bytes + 7u) / 8u * 8u;
     pl.smem = 1024 + pl.bar_off + 2 * kLaMaxStages * sizeof(uint64_t);
-    // the first stages into L2 before the dependency wait
-    pl.pf_stages = S;
+    // L2 prefetch of the first stages before the dependency wait, only when
+    // the ring is shorter than K: otherwise every stage's copy is issued at
+    // once right after the wait, and issuing the prefetches first would only
+    // delay those copies
+    pl.pf_stages = S < pl.num_kb ? S : 0;
     return true;
+}
+
+bool plan_la(const WeightView& w, int mode, LaPlan& pl) {
+    const DeviceInfo& dev = device_info();
+    if (w.N < 1 || w.K < 16 || w.K % 16 != 0 || w.K > 32768 || w.N > (1 << 30)) return false;
+    if (w.gs != 16 && w.gs != 32 && w.gs != 64 && w.gs != 128) return false;
+    if (w.G % 8 != 0) return false;  // table rows must be 16-byte multiples for the tensor copies
+    const int64_t sms = dev.sm_count;
+    if ((w.N + sms - 1) / sms > kLaMaxPairs * 16) return false;  // at most 128 rows per SM, one CTA per SM
+    const int R = static_cast<int>((w.N + sms - 1) / sms);
+    const int npair = (R + 15) / 16;
+    // Codes per stage: fewer, larger stages mean fewer stage synchronisations
+    // and one scale/bias load for two chunks, as long as the ring stays deep
+    // enough: 2048 codes for up to two tiles when all of K fits in the ring,
+    // 1024 for up to four tiles, 512 above (group size 128 needs >= 1024).
+    const size_t budget = static_cast<size_t>(dev.max_smem_optin);
+    if (npair <= 2 && kLaCpl4 && plan_geometry(w, mode, R, 4, budget, 1, pl) && pl.S == pl.num_kb) return true;
+    const int cpl = (w.gs == 128 || npair <= 4) ? 2 : 1;
+    return plan_geometry(w, mode, R, cpl, budget, 1, pl);
 }
 
 }  // namespace
@@ -397,7 +447,9 @@ cudaError_t launch_gemv_la(const WeightView& w, int mode, const void* x, const v
     p.S = pl.S;
     p.gpk = pl.gpk;
     p.Kpad = pl.Kpad;
-    p.pf_stages = pl.pf_stages;
+    // a static weight: the ring's first stages are copied before the dependency wait
+    p.pre_wait = (w.flags & MLXQ_WEIGHT_STATIC) ? pl.S : 0;
+    p.pf_stages = (w.flags & MLXQ_WEIGHT_STATIC) ? 0 : pl.pf_stages;
     p.box_bytes = pl.box_bytes;
     p.sb_bytes = pl.sb_bytes;
     p.stage_bytes = pl.stage_bytes;

@@ -18,6 +18,7 @@ struct WeightView {
     const uint16_t* scales;  // [N, G] bf16 bits
     const uint16_t* biases;  // [N, G] bf16 bits
     int64_t N, K, gs, G;
+    uint32_t flags;          // MLXQ_WEIGHT_*
 };
 
 enum GemvMode { GEMV_PLAIN = 0, GEMV_SILU = 1, GEMV_SILU_RESID = 2 };
@@ -93,6 +94,11 @@ bool stream_mma_supported(const WeightView& w, int mode, int64_t m, const void* 
                           const void* up);
 cudaError_t launch_stream_mma(const WeightView& w, int mode, int64_t m, const void* x, const void* gate,
                               const void* up, const void* resid, void* y, cudaStream_t stream);
+
+// Small-m gemm, 1 <= m <= 32, weight tiles walked in groups by one CTA per
+// SM (tensor-pipe fragments, activations copied with each stage).
+bool smallm_supported(const WeightView& w, int64_t m, const void* X);
+cudaError_t launch_smallm(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream);
 
 // CUDA-core small-m gemm: Y [m, N] = X [m, K] W^T, 2 <= m <= kSmallMMax.
 constexpr int kSmallMMax = 32;
