@@ -182,9 +182,13 @@ enum {
     MLXQ_GEMM_AUTO = 0,        /* what mlxq_gemm picks */
     MLXQ_GEMM_ROWS = 1,        /* m independent passes of the gemv kernel */
     MLXQ_GEMM_SMALLM = 2,      /* weight-streaming kernel, products on the tensor pipe
-                                  (mma.sync fragments), m <= 32 */
+                                  (mma.sync fragments), m <= 32: each CTA streams its
+                                  rows in pairs of 8-row octets */
     MLXQ_GEMM_TCGEN05 = 3,     /* tcgen05 tensor-core kernel (TMEM accumulators) */
-    MLXQ_GEMM_SMALLM_FFMA = 4  /* weight-streaming kernel on the fp32 pipes, m <= 32 */
+    MLXQ_GEMM_SMALLM_FFMA = 4, /* weight-streaming kernel on the fp32 pipes, m <= 32 */
+    MLXQ_GEMM_SMALLM_GROUPS = 5 /* weight-streaming kernel on the tensor pipe, m <= 32:
+                                  each SM walks a balanced range of 16-row tiles in
+                                  groups; in_features % 128 == 0, group_size 16/32/64 */
 };
 
 /* mlxq_gemm with an explicit kernel; MLXQ_ERR_UNSUPPORTED if that kernel

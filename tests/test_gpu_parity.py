@@ -442,6 +442,31 @@ def test_gemm_smallm_tensor_pipe(N, K, gs, m):
     assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_AUTO), ref, f"auto m={m} {N}x{K}")
 
 
+# the tile-group kernel wants K % 128 == 0 and gs in {16, 32, 64}; the rows
+# per CTA span one partial group, one or several full groups, and a ragged
+# last tile
+GROUP_SHAPES = [(512, 1024, 64), (300, 4096, 32), (77, 512, 16), (5000, 1152, 16), (2100, 2304, 32),
+                (14336 + 8, 512, 64), (4096, 384, 16)]
+
+
+@pytest.mark.parametrize("N,K,gs", GROUP_SHAPES)
+@pytest.mark.parametrize("m", [1, 2, 7, 8, 9, 16, 17, 31, 32])
+def test_gemm_smallm_tile_groups(N, K, gs, m):
+    W, g = make(11, N, K, gs)
+    X = synth.activations(g, m, K)
+    ref = oracle.gemm(*W.host, gs, X)
+    assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_SMALLM_GROUPS), ref, f"smallm-groups m={m} {N}x{K}")
+
+
+def test_gemm_smallm_tile_groups_refuses_what_it_cannot_take():
+    W, g = make(12, 256, 14336, 128)  # gs = 128: not taken
+    X = dev(synth.activations(g, 4, 14336))
+    Y = torch.empty(4 * 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(mq.MlxqError) as e:
+        mq.mlxq_gemm_with(W.w, X, Y.data_ptr(), 4, mq.MLXQ_GEMM_SMALLM_GROUPS)
+    assert e.value.code == mq.MLXQ_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("N,K,gs", SMALLM_SHAPES + [(300, 4096, 256)])
 @pytest.mark.parametrize("m", [1, 2, 4, 5, 16, 32])
 def test_gemm_smallm_fp32_pipes(N, K, gs, m):

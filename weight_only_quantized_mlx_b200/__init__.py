@@ -35,6 +35,7 @@ MLXQ_GEMM_ROWS = 1
 MLXQ_GEMM_SMALLM = 2
 MLXQ_GEMM_TCGEN05 = 3
 MLXQ_GEMM_SMALLM_FFMA = 4
+MLXQ_GEMM_SMALLM_GROUPS = 5
 
 MLXQ_WEIGHT_STATIC = 1
 

@@ -598,7 +598,7 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
     WeightView v;
     int rc = check_weight(w, v);
     if (rc) return rc;
-    if (kernel < MLXQ_GEMM_AUTO || kernel > MLXQ_GEMM_SMALLM_FFMA)
+    if (kernel < MLXQ_GEMM_AUTO || kernel > MLXQ_GEMM_SMALLM_GROUPS)
         return fail(MLXQ_ERR_INVALID_ARG, "unknown gemm kernel id %d", kernel);
     if (m == 0) return ok();
     const int64_t M = m;
@@ -614,8 +614,10 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
     int k = kernel;
     if (k == MLXQ_GEMM_AUTO) {
         if (M == 1) k = MLXQ_GEMM_ROWS;
+        else if (M <= kStreamMmaMaxM && smallm_preferred(v, M, x)) k = MLXQ_GEMM_SMALLM_GROUPS;
         else if (M <= kStreamMmaMaxM && stream_mma_supported(v, GEMV_PLAIN, M, x, nullptr, nullptr))
             k = MLXQ_GEMM_SMALLM;
+        else if (smallm_supported(v, M, x)) k = MLXQ_GEMM_SMALLM_GROUPS;
         else if (gemm_tc_supported(v, M, x, y)) k = MLXQ_GEMM_TCGEN05;
         else if (M <= kSmallMMax && x16 && gemm_smallm_supported(v, M)) k = MLXQ_GEMM_SMALLM_FFMA;
         else k = MLXQ_GEMM_ROWS;
@@ -630,6 +632,11 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
             }
             return ok();
         }
+        case MLXQ_GEMM_SMALLM_GROUPS:
+            if (!smallm_supported(v, M, x))
+                return fail(MLXQ_ERR_UNSUPPORTED, "small-m tile-group kernel cannot take m=%lld, K=%lld, group_size=%lld",
+                            static_cast<long long>(M), static_cast<long long>(v.K), static_cast<long long>(v.gs));
+            return launch_status(launch_smallm(v, x, y, M, s), "small-m tile-group gemm launch");
         case MLXQ_GEMM_SMALLM:
             if (M > kStreamMmaMaxM || !stream_mma_supported(v, GEMV_PLAIN, M, x, nullptr, nullptr))
                 return fail(MLXQ_ERR_UNSUPPORTED, "small-m tensor-pipe kernel cannot take m=%lld, K=%lld, group_size=%lld",

@@ -98,6 +98,9 @@ cudaError_t launch_stream_mma(const WeightView& w, int mode, int64_t m, const vo
 // Small-m gemm, 1 <= m <= 32, weight tiles walked in groups by one CTA per
 // SM (tensor-pipe fragments, activations copied with each stage).
 bool smallm_supported(const WeightView& w, int64_t m, const void* X);
+// supported, and measured faster than the per-row-pair streaming kernel:
+// 8 < m and at least 6 tiles of 16 rows per SM
+bool smallm_preferred(const WeightView& w, int64_t m, const void* X);
 cudaError_t launch_smallm(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream);
 
 // CUDA-core small-m gemm: Y [m, N] = X [m, K] W^T, 2 <= m <= kSmallMMax.

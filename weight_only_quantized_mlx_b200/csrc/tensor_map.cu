@@ -45,6 +45,19 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint6
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_3d_chunks(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_bytes, const void* base, uint64_t inner,
+                      uint64_t outer, uint64_t row_bytes, uint32_t chunk, uint32_t box_outer, uint32_t box_chunks) {
+    auto enc = encoder();
+    if (!enc || chunk == 0 || inner % chunk != 0) return false;
+    const cuuint64_t dims[3] = {chunk, outer, inner / chunk};
+    const cuuint64_t strides[2] = {row_bytes, static_cast<cuuint64_t>(chunk) * elem_bytes};
+    const cuuint32_t box[3] = {chunk, box_outer, box_chunks};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool weight_tensor_maps(const WeightView& w, int box_rows, int box_k_bytes, CUtensorMapSwizzle packed_sw,
                         int box_groups, TensorMaps3* out) {
     int dev = 0;

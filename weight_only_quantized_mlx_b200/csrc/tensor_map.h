@@ -23,6 +23,14 @@ bool tensor_maps_available();
 bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 
+// 3-D tiled map over a row-major [outer, inner] array viewed as
+// {chunk, outer, inner / chunk} (strides row_bytes and chunk * elem bytes),
+// so that one box {chunk, box_outer, box_chunks} brings box_chunks
+// consecutive chunks of box_outer rows, chunk-major in shared memory
+// ([box_chunks][box_outer][chunk]); 128-byte swizzle, zero fill out of bounds.
+bool encode_3d_chunks(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_bytes, const void* base, uint64_t inner,
+                      uint64_t outer, uint64_t row_bytes, uint32_t chunk, uint32_t box_outer, uint32_t box_chunks);
+
 // Maps of a weight: packed box {box_k_bytes, box_rows} with swizzle
 // `packed_sw`; scale/bias boxes {box_groups, box_rows} (box_groups == 0: no
 // scale/bias maps).  Returns false if encoding failed.
