@@ -83,8 +83,8 @@ typedef struct mlxq_weight {
  * MLXQ_WEIGHT_STATIC: the caller guarantees that while a call that reads this
  * weight is queued or running, no kernel on any stream writes its packed,
  * scales or biases buffers (true of weights loaded once and then only read,
- * as in decoding).  The m = 1 kernels may then copy the weight into shared
- * memory before the previous work on the stream has finished; activations,
+ * as in decoding).  The m = 1 kernels and dequantize_to may then read the
+ * weight before the previous work on the stream has finished; activations,
  * residuals and outputs are still touched only after it.  Off (0) by default:
  * every read of the weight then comes after the previous work on the stream.
  */

@@ -81,6 +81,16 @@ def test_dequant_misaligned_output_takes_generic_path():
     assert np.array_equal(out.value_bits(), oracle.dequant(*W.host, 32).ravel())
 
 
+@pytest.mark.parametrize("offset_elems", [8, 16])  # 16-byte aligned only; 32-byte aligned
+def test_dequant_vector_paths_by_output_alignment(offset_elems):
+    W, _ = make(3, 300, 1024 + 64, 64)  # several block steps and a ragged last one
+    out = Guarded(300 * 1088, offset_elems=offset_elems)
+    mq.mlxq_dequant(W.w, out.data_ptr())
+    torch.cuda.synchronize()
+    out.check_guards()
+    assert np.array_equal(out.value_bits(), oracle.dequant(*W.host, 64).ravel())
+
+
 def test_dequant_decode_workload_100_pairs():
     out = torch.empty(4096 * 4096, dtype=torch.bfloat16, device="cuda")
     for seed in range(100):

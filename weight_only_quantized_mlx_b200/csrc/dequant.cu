@@ -7,6 +7,7 @@
 // result is bit-identical to any correct fp32 implementation of the formula.
 #include <cuda_fp16.h>
 
+#include <atomic>
 #include <cstring>
 
 #include "device_common.cuh"
@@ -16,38 +17,76 @@ namespace mlxq {
 namespace {
 
 // Fast path: K % 16 == 0, group_size % 16 == 0, 16-byte aligned buffers.
-// One thread per 16-code chunk; a chunk never straddles a group.
+// A chunk is 16 codes (one 16-byte load, 32 bytes stored) and never
+// straddles a group.  Each block owns a balanced contiguous range of chunks
+// and walks it kDqU * 256 chunks per step; a thread issues all kDqU loads
+// (and their table loads) before its first store, so each SM keeps enough
+// bytes in flight to cover HBM latency.
+// The grid is one resident wave and is launched as a programmatic dependent:
+// the output is written only after the previous kernel on the stream has
+// finished; a weight marked static is also read before that point.
+// V8: the output is 32-byte aligned and each chunk is one 32-byte store
+// (whole sectors); otherwise two 16-byte stores.
+constexpr int kDqU = 4;
+template <bool V8>
 __global__ void __launch_bounds__(256) k_dequant_vec16(const uint4* __restrict__ packed,
                                                        const uint16_t* __restrict__ scales,
                                                        const uint16_t* __restrict__ biases,
-                                                       uint4* __restrict__ out, int64_t nchunks,
-                                                       int64_t chunks_per_row,
-                                                       int64_t chunks_per_group, int64_t G) {
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < nchunks;
-         c += stride) {
-        const int64_t n = c / chunks_per_row;
-        const int64_t j = c - n * chunks_per_row;
-        const int64_t gi = n * G + j / chunks_per_group;
-        const uint4 wq = ldg_nc_v4(packed + c);
-        const float s = bf16_bits_to_f32(__ldg(scales + gi));
-        const float b = bf16_bits_to_f32(__ldg(biases + gi));
-        const uint32_t words[4] = {wq.x, wq.y, wq.z, wq.w};
-        uint32_t o[8];
+                                                       uint4* __restrict__ out, uint32_t nchunks,
+                                                       uint32_t chunks_per_row, uint32_t chunks_per_group,
+                                                       uint32_t G, int pre_wait) {
+    pdl_launch_dependents();
+    bool waited = pre_wait == 0;
+    if (waited) pdl_wait();
+    // this block's share: a balanced contiguous range of chunks
+    const uint64_t lo = static_cast<uint64_t>(nchunks) * blockIdx.x / gridDim.x;
+    const uint64_t hi = static_cast<uint64_t>(nchunks) * (blockIdx.x + 1) / gridDim.x;
+    for (uint64_t base = lo; base < hi; base += kDqU * 256u) {
+        uint4 wq[kDqU];
+        float s[kDqU], b[kDqU];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t w = words[i];
-            const float q0 = code_magic<0>(w) - kMagic;
-            const float q1 = code_magic<1>(w) - kMagic;
-            const float q2 = code_magic<2>(w) - kMagic;
-            const float q3 = code_magic<3>(w) - kMagic;
-            o[2 * i] = pack_bf16x2(__fmaf_rn(s, q0, b), __fmaf_rn(s, q1, b));
-            o[2 * i + 1] = pack_bf16x2(__fmaf_rn(s, q2, b), __fmaf_rn(s, q3, b));
+        for (int u = 0; u < kDqU; ++u) {
+            const uint64_t c = base + u * 256u + threadIdx.x;
+            if (c < hi) {
+                const uint32_t n = static_cast<uint32_t>(c) / chunks_per_row;
+                const uint32_t j = static_cast<uint32_t>(c) - n * chunks_per_row;
+                const uint64_t gi = static_cast<uint64_t>(n) * G + j / chunks_per_group;
+                wq[u] = ldg_nc_v4(packed + c);
+                s[u] = bf16_bits_to_f32(__ldg(scales + gi));
+                b[u] = bf16_bits_to_f32(__ldg(biases + gi));
+            }
         }
-        uint4* dst = out + 2 * c;
-        __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
-        __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+        if (!waited) {
+            pdl_wait();
+            waited = true;
+        }
+#pragma unroll
+        for (int u = 0; u < kDqU; ++u) {
+            const uint64_t c = base + u * 256u + threadIdx.x;
+            if (c < hi) {
+                const uint32_t words[4] = {wq[u].x, wq[u].y, wq[u].z, wq[u].w};
+                uint32_t o[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w = words[i];
+                    const float q0 = code_magic<0>(w) - kMagic;
+                    const float q1 = code_magic<1>(w) - kMagic;
+                    const float q2 = code_magic<2>(w) - kMagic;
+                    const float q3 = code_magic<3>(w) - kMagic;
+                    o[2 * i] = pack_bf16x2(__fmaf_rn(s[u], q0, b[u]), __fmaf_rn(s[u], q1, b[u]));
+                    o[2 * i + 1] = pack_bf16x2(__fmaf_rn(s[u], q2, b[u]), __fmaf_rn(s[u], q3, b[u]));
+                }
+                uint4* dst = out + 2ull * c;
+                if constexpr (V8) {
+                    stg_cs_v8(dst, o);
+                } else {
+                    __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+                    __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+                }
+            }
+        }
     }
+    if (!waited) pdl_wait();
 }
 
 // Any shape the format allows (K % 4 == 0, any group_size dividing K, any
@@ -131,15 +170,28 @@ cudaError_t launch_dequant(const WeightView& w, void* out, cudaStream_t stream) 
     if (total == 0) return cudaSuccess;
     const int sms = device_info().sm_count;
     const bool vec = (w.K % 16 == 0) && (w.gs % 16 == 0) && aligned16(w.packed) &&
-                     aligned16(out);
+                     aligned16(out) && total / 16 < (int64_t{1} << 32) && w.G < (int64_t{1} << 32);
     if (vec) {
         const int64_t nchunks = total / 16;
-        int64_t blocks = (nchunks + 255) / 256;
-        const int64_t cap = static_cast<int64_t>(sms) * 32;
-        if (blocks > cap) blocks = cap;
-        k_dequant_vec16<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            reinterpret_cast<const uint4*>(w.packed), w.scales, w.biases,
-            reinterpret_cast<uint4*>(out), nchunks, w.K / 16, w.gs / 16, w.G);
+        const int64_t tiles = (nchunks + kDqU * 256 - 1) / (kDqU * 256);
+        const bool v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+        auto kern = v8 ? k_dequant_vec16<true> : k_dequant_vec16<false>;
+        static std::atomic<int> per_sm[2];  // resident blocks per SM, asked once per variant
+        if (per_sm[v8].load() == 0) {
+            int b = 0;
+            cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, 256, 0);
+            if (e != cudaSuccess) return e;
+            per_sm[v8].store(b > 0 ? b : 1);
+        }
+        const int64_t wave = static_cast<int64_t>(sms) * per_sm[v8].load();  // one resident wave
+        const int blocks = static_cast<int>(tiles < wave ? tiles : wave);
+        const int pre_wait = (w.flags & MLXQ_WEIGHT_STATIC) ? 1 : 0;
+        cudaError_t e = launch_pdl(kern, dim3(blocks), dim3(256), 0, stream,
+                                   reinterpret_cast<const uint4*>(w.packed), w.scales, w.biases,
+                                   reinterpret_cast<uint4*>(out), static_cast<uint32_t>(nchunks),
+                                   static_cast<uint32_t>(w.K / 16), static_cast<uint32_t>(w.gs / 16),
+                                   static_cast<uint32_t>(w.G), pre_wait);
+        if (e != cudaSuccess) return e;
     } else {
         const int64_t nwords = total / 4;
         int64_t blocks = (nwords + 255) / 256;

@@ -172,6 +172,13 @@ __device__ __forceinline__ uint16_t lds16(uint32_t addr) {
     return v;
 }
 
+// One 32-byte streaming store (a full sector per thread; 32-byte aligned).
+__device__ __forceinline__ void stg_cs_v8(void* p, const uint32_t (&v)[8]) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
