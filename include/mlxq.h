@@ -185,7 +185,10 @@ enum {
                                   (mma.sync fragments), m <= 32: each CTA streams its
                                   rows in pairs of 8-row octets */
     MLXQ_GEMM_TCGEN05 = 3,     /* tcgen05 tensor-core kernel (TMEM accumulators) */
-    MLXQ_GEMM_SMALLM_FFMA = 4, /* weight-streaming kernel on the fp32 pipes, m <= 32 */
+    MLXQ_GEMM_SMALLM_FFMA = 4, /* weight-streaming kernel on the fp32 pipes: m <= 32
+                                  when group_size % 16 == 0; any m, in passes of up to
+                                  8 rows, for other group sizes with group_size % 4 == 0
+                                  and in_features % 16 == 0 */
     MLXQ_GEMM_SMALLM_GROUPS = 5 /* weight-streaming kernel on the tensor pipe, m <= 32:
                                   each SM walks a balanced range of 16-row tiles in
                                   groups; in_features % 128 == 0, group_size 16/32/64 */

@@ -619,7 +619,8 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
             k = MLXQ_GEMM_SMALLM;
         else if (smallm_supported(v, M, x)) k = MLXQ_GEMM_SMALLM_GROUPS;
         else if (gemm_tc_supported(v, M, x, y)) k = MLXQ_GEMM_TCGEN05;
-        else if (M <= kSmallMMax && x16 && gemm_smallm_supported(v, M)) k = MLXQ_GEMM_SMALLM_FFMA;
+        else if ((M <= kSmallMMax && x16 && gemm_smallm_supported(v, M)) || anygs_gemm_supported(v, M))
+            k = MLXQ_GEMM_SMALLM_FFMA;
         else k = MLXQ_GEMM_ROWS;
     }
     switch (k) {
@@ -644,10 +645,14 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
             return launch_status(launch_stream_mma(v, GEMV_PLAIN, M, x, nullptr, nullptr, nullptr, y, s),
                                  "small-m gemm launch");
         case MLXQ_GEMM_SMALLM_FFMA:
-            if (!gemm_smallm_supported(v, M) || !x16)
+            if (M <= kSmallMMax && x16 && gemm_smallm_supported(v, M))
+                return launch_status(launch_gemm_smallm(v, x, y, M, s), "small-m fp32 gemm launch");
+            if (anygs_gemm_supported(v, M))
+                return launch_status(launch_anygs_gemm(v, x, y, M, s), "small-m fp32 gemm (any group size) launch");
+            {
                 return fail(MLXQ_ERR_UNSUPPORTED, "small-m fp32 kernel cannot take m=%lld, K=%lld, group_size=%lld",
                             static_cast<long long>(M), static_cast<long long>(v.K), static_cast<long long>(v.gs));
-            return launch_status(launch_gemm_smallm(v, x, y, M, s), "small-m fp32 gemm launch");
+            }
         default:
             if (!gemm_tc_supported(v, M, x, y))
                 return fail(MLXQ_ERR_UNSUPPORTED, "tensor-core kernel cannot take m=%lld, N=%lld, K=%lld, group_size=%lld",

@@ -192,6 +192,8 @@ cudaError_t launch_dequant(const WeightView& w, void* out, cudaStream_t stream) 
                                    static_cast<uint32_t>(w.K / 16), static_cast<uint32_t>(w.gs / 16),
                                    static_cast<uint32_t>(w.G), pre_wait);
         if (e != cudaSuccess) return e;
+    } else if (anygs_dequant_supported(w, out)) {
+        return launch_anygs_dequant(w, out, stream);
     } else {
         const int64_t nwords = total / 4;
         int64_t blocks = (nwords + 255) / 256;

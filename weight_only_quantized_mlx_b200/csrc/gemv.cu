@@ -408,6 +408,7 @@ cudaError_t launch_gemv(const WeightView& w, int mode, const void* x, const void
     p.resid = static_cast<const uint16_t*>(resid);
     p.y = static_cast<uint16_t*>(y);
     p.i0 = 0;
+    if (!pl.vec && anygs_gemv_supported(w, mode)) return launch_anygs_gemv(w, mode, x, gate, up, resid, y, stream);
     if (!pl.vec) {
         const int sms = device_info().sm_count;
         const int64_t blocks64 = (w.N + 7) / 8;

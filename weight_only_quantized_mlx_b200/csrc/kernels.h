@@ -103,6 +103,16 @@ bool smallm_supported(const WeightView& w, int64_t m, const void* X);
 bool smallm_preferred(const WeightView& w, int64_t m, const void* X);
 cudaError_t launch_smallm(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream);
 
+// Any group size with 4-code words (gs % 4 == 0, K % 16 == 0, 16-byte
+// aligned codes; tables and activations need only 2-byte alignment).
+bool anygs_gemv_supported(const WeightView& w, int mode);
+cudaError_t launch_anygs_gemv(const WeightView& w, int mode, const void* x, const void* gate, const void* up,
+                              const void* resid, void* y, cudaStream_t stream);
+bool anygs_gemm_supported(const WeightView& w, int64_t m);
+cudaError_t launch_anygs_gemm(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream);
+bool anygs_dequant_supported(const WeightView& w, const void* out);  // out 16-byte aligned
+cudaError_t launch_anygs_dequant(const WeightView& w, void* out, cudaStream_t stream);
+
 // CUDA-core small-m gemm: Y [m, N] = X [m, K] W^T, 2 <= m <= kSmallMMax.
 constexpr int kSmallMMax = 32;
 bool gemm_smallm_supported(const WeightView& w, int64_t m);
