@@ -382,6 +382,32 @@ def measure_rows(mq, torch, synth, dev, stream, dec_weights, peaks, args):
     qdst.release()
     del qsrc
 
+    # a group size the tensor-pipe kernels do not take (8: any-group-size
+    # kernels) on the decode shape; 16 weights of 25 MB rotate (400 MB, more
+    # than L2)
+    gs8 = 8
+    w8 = [upload_weight(mq, *synth.weight(synth.rng(7000 + i), D_N, D_K, gs8), gs8) for i in range(16)]
+    x8 = torch.randn(D_K, device=dev).to(torch.bfloat16)
+    y8 = torch.empty(D_N, dtype=torch.bfloat16, device=dev)
+    ms = time_region(lambda: [mq.mlxq_gemv(w.handle, x8, y8, stream) for w in w8], steps, warm, stream, 1)
+    b = gemv_bytes(D_N, D_K, gs8) * len(w8)
+    gbs = b / (ms * 1e-3) / 1e9
+    rows["gemv_4096x4096_gs8"] = {"value": round(gbs, 1), "unit": "GB/s", "frac_hbm": round(gbs / hbm, 4),
+                                  "us_per_launch": round(ms * 1e3 / len(w8), 2), "kernel": "k_anygs_gemv"}
+    outs = [torch.empty(D_N * D_K, dtype=torch.bfloat16, device=dev) for _ in range(8)]
+
+    def deq8():
+        for i, w in enumerate(w8):
+            mq.mlxq_dequant(w.handle, outs[i % len(outs)], stream)
+    ms = time_region(deq8, steps, warm, stream, 1)
+    b = (D_N * D_K + 4 * D_N * D_K // gs8 + 2 * D_N * D_K) * len(w8)
+    gbs = b / (ms * 1e-3) / 1e9
+    rows["dequant_4096x4096_gs8"] = {"value": round(gbs, 1), "unit": "GB/s", "frac_hbm": round(gbs / hbm, 4),
+                                     "kernel": "k_dequant_anygs"}
+    del outs
+    for w in w8:
+        w.release()
+
     # fused decode MLP: gate, up (14336x4096) then silu_gate_resid down (4096x14336)
     D, F, gs = 4096, 14336, 64
     mlps = []
