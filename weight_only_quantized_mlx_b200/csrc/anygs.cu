@@ -69,16 +69,47 @@ __global__ void __launch_bounds__(kAgThreads) k_anygs_gemv(const AgParams p) {
     // activations: plain -> BF16 [MT][K]; silu -> fp32 h [K]
     pdl_launch_dependents();
     pdl_wait();
+    // (16-byte loads when the vectors are 16-byte aligned, K % 16 == 0 keeping
+    // every row aligned; several loads in flight per thread either way)
     if (MODE == GEMV_PLAIN) {
-        uint16_t* xs = reinterpret_cast<uint16_t*>(smem_ag);
-        for (int e = threadIdx.x; e < MT * K; e += kAgThreads) {
-            const int i = e / K, k = e - i * K;
-            xs[e] = (i < p.mt) ? p.x[static_cast<int64_t>(p.i0 + i) * K + k] : uint16_t(0);
+        if ((reinterpret_cast<uintptr_t>(p.x) & 15u) == 0) {
+            uint4* xs = reinterpret_cast<uint4*>(smem_ag);
+            const int k8 = K / 8;
+#pragma unroll 4
+            for (int e = threadIdx.x; e < MT * k8; e += kAgThreads) {
+                const int i = e / k8, c = e - i * k8;
+                xs[e] = (i < p.mt) ? ldg_nc_v4(p.x + static_cast<int64_t>(p.i0 + i) * K + 8 * c)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            }
+        } else {
+            uint16_t* xs = reinterpret_cast<uint16_t*>(smem_ag);
+#pragma unroll 8
+            for (int e = threadIdx.x; e < MT * K; e += kAgThreads) {
+                const int i = e / K, k = e - i * K;
+                xs[e] = (i < p.mt) ? p.x[static_cast<int64_t>(p.i0 + i) * K + k] : uint16_t(0);
+            }
         }
     } else {
         float* hs = reinterpret_cast<float*>(smem_ag);
-        for (int k = threadIdx.x; k < K; k += kAgThreads)
-            hs[k] = silu_ag(bf16_bits_to_f32(p.gate[k])) * bf16_bits_to_f32(p.up[k]);
+        if (((reinterpret_cast<uintptr_t>(p.gate) | reinterpret_cast<uintptr_t>(p.up)) & 15u) == 0) {
+#pragma unroll 2
+            for (int c = threadIdx.x; c < K / 8; c += kAgThreads) {
+                const uint4 gv = ldg_nc_v4(p.gate + 8 * c), uv = ldg_nc_v4(p.up + 8 * c);
+                const uint32_t gg[4] = {gv.x, gv.y, gv.z, gv.w}, uu[4] = {uv.x, uv.y, uv.z, uv.w};
+                float h[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    h[2 * i] = silu_ag(bf16_bits_to_f32(gg[i] & 0xFFFFu)) * bf16_bits_to_f32(uu[i] & 0xFFFFu);
+                    h[2 * i + 1] = silu_ag(bf16_bits_to_f32(gg[i] >> 16)) * bf16_bits_to_f32(uu[i] >> 16);
+                }
+                reinterpret_cast<float4*>(hs)[2 * c] = make_float4(h[0], h[1], h[2], h[3]);
+                reinterpret_cast<float4*>(hs)[2 * c + 1] = make_float4(h[4], h[5], h[6], h[7]);
+            }
+        } else {
+#pragma unroll 8
+            for (int k = threadIdx.x; k < K; k += kAgThreads)
+                hs[k] = silu_ag(bf16_bits_to_f32(p.gate[k])) * bf16_bits_to_f32(p.up[k]);
+        }
     }
     __syncthreads();
 

@@ -5,7 +5,9 @@
 // to nearest even,
 //   lo, hi = min, max;  s = bf16((hi - lo) / 255);  b = bf16(lo);
 //   q = clamp(rint((w - b) / s), 0, 255)   (q = 0 when s == 0).
-// HBM-bound: 2 bytes read and 1 + 4/gs bytes written per weight.
+// HBM-bound: 2 bytes read and 1 + 4/gs bytes written per weight.  The
+// quotient is computed approximately and made exact only near a tie, so the
+// codes equal those of the correctly rounded division.
 //
 // k_quantize_lanes (gs = 8..256, a power of two, 16-byte aligned source):
 // gs/8 consecutive lanes share a group, each loading 8 BF16 (16 bytes,
@@ -112,11 +114,25 @@ __global__ void __launch_bounds__(256) k_quantize_lanes(const uint16_t* __restri
     const __nv_bfloat16 bb = __float2bfloat16_rn(lo);
     const float sf = __bfloat162float(sb), bf = __bfloat162float(bb);
     uint32_t word[2] = {0u, 0u};
+    // An approximate quotient rounds to the same integer as the correctly
+    // rounded one unless it lies within a few ulps of a half-integer; there,
+    // and for operands outside the range where the approximation holds, the
+    // correctly rounded division decides.
+    const float as = fabsf(sf);
+    const bool fast_ok = as > 0x1p-100f && as < 0x1p100f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         float c = 0.0f;
         if (sf != 0.0f) {
-            c = rintf(__fdiv_rn(__fsub_rn(f[i], bf), sf));
+            const float d = __fsub_rn(f[i], bf);
+            float qv;
+            if (fast_ok && fabsf(d) < 0x1p100f) {
+                qv = __fdividef(d, sf);
+                if (fabsf(qv - floorf(qv) - 0.5f) < 0x1p-10f) qv = __fdiv_rn(d, sf);
+            } else {
+                qv = __fdiv_rn(d, sf);
+            }
+            c = rintf(qv);
             if (c < 0.0f) c = 0.0f;
             if (c > 255.0f) c = 255.0f;
         }
