@@ -591,6 +591,31 @@ def test_gemm_tcgen05_split_k(N, K, gs, m):
     assert np.array_equal(y1, y2)
 
 
+# More tiles than SMs with a partial last wave: whole tiles fill the full
+# waves and the last wave's tiles split K over the SMs it would leave idle.
+# (N, K, gs, m) -> tiles: 149 (1 split tile), 160 (12 split tiles, BN 256),
+# 151 with a ragged last weight tile and ragged m.
+TC_TAIL_SHAPES = [
+    (256 * 149, 1024, 64, 32),
+    (256 * 40, 1024, 32, 1024),
+    (256 * 150 + 77, 2048, 128, 40),
+]
+
+
+@pytest.mark.parametrize("N,K,gs,m", TC_TAIL_SHAPES)
+def test_gemm_tcgen05_tail_split(N, K, gs, m):
+    W, g = make(42, N, K, gs)
+    X = synth.activations(g, m, K)
+    y1 = run_gemm(W, X, m, mq.MLXQ_GEMM_TCGEN05)
+    y2 = run_gemm(W, X, m, mq.MLXQ_GEMM_TCGEN05)
+    assert np.array_equal(y1, y2)  # split tiles are summed in split order
+    pick_w = np.unique(np.concatenate([tile_edges(N, 256), np.arange(N - 300, N),
+                                       np.random.default_rng(N).choice(N, 64, replace=False)]))
+    pick_x = np.unique(np.concatenate([tile_edges(m, 256), np.random.default_rng(m).choice(m, min(m, 24), replace=False)]))
+    ref = oracle.gemm(*rows_subset(W, pick_w), gs, X[pick_x])
+    assert_close(y1[np.ix_(pick_x, pick_w)], ref, f"tc tail {N}x{K}/{gs} m={m}")
+
+
 def test_gemm_tcgen05_integer_weights_exact():
     # s = 1, b = 0 and small-integer X: every BF16 product and fp32 partial sum is
     # an exact integer below 2^24, so the tensor-core result must equal the

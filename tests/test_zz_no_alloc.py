@@ -71,6 +71,20 @@ def test_noalloc_matches_gemm_and_oracle(N, K, gs, m):
     assert_close(y_na, oracle.gemm(*host, gs, X_bits), f"noalloc {N}x{K}/{gs} m={m}")
 
 
+def test_noalloc_tail_split_matches_gemm():
+    # 149 tiles: the last wave's tile splits K; both calls take the same plan
+    N, K, gs, m = 256 * 149, 1024, 64, 32 + 8
+    host, keep, w, g = weight(79, N, K, gs)
+    X_bits = synth.activations(g, m, K)
+    X = dev(X_bits)
+    y_na = call(mq.mlxq_gemm_noalloc, w, X, m, N)
+    y_ref = call(mq.mlxq_gemm, w, X, m, N)
+    assert np.array_equal(y_na, y_ref)
+    rows = np.concatenate([np.arange(0, 40), np.arange(N - 256, N)])
+    p, s, b = host
+    assert_close(y_na[:, rows], oracle.gemm(p[rows], s[rows], b[rows], gs, X_bits), "noalloc tail split")
+
+
 def test_noalloc_two_calls_in_a_row():
     # different shapes, back to back on one stream with no synchronisation
     ha, keep_a, wa, ga = weight(80, 512, 4096, 64)  # keep_*: the device arrays the views point at

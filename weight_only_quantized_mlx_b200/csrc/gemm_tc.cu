@@ -18,10 +18,11 @@
 //   warps 11-18 after a unit's last k-block, read the accumulators
 //               (tcgen05.ld) and store Y (or the unit's fp32 partial)
 //
-// When the tiles alone would leave SMs idle, each tile's K is split over
-// several CTAs: each stores its fp32 partial tile, and the last to finish
-// (a per-tile counter) adds them in split order, so the result does not
-// depend on which CTA finishes when.  The accumulator is D[w_row][x_row]
+// When the tiles alone would leave SMs idle (fewer tiles than SMs, or the
+// tiles of a partial last wave), those tiles' K is split over several CTAs:
+// each stores its fp32 partial tile, and the last to finish (a per-tile
+// counter) adds them in split order, so the result does not depend on which
+// CTA finishes when.  The tiles of the full waves stay whole.  The accumulator is D[w_row][x_row]
 // (TMEM lane = weight row), so a warp's stores of one output row of Y are 32
 // consecutive BF16 values.  All pipeline waits are bounded; no cluster
 // multicast is used.  After a wait gives up, the producers and the MMA thread
@@ -63,9 +64,11 @@ struct TcParams {
     int BN, S, SX, num_kb;  // S: A-tile stages, SX: activation-tile stages
     int sg;          // k-blocks covered by one scale/bias box (8 * gs / 64)
     int sb_tma;      // 1: scales/biases by TMA boxes; 0 (rows not 16-byte multiples): direct loads
-    int ks;          // K splits per tile (1: no split)
-    float* ws;       // ks > 1: fp32 partial tiles [tiles * ks][BN][kBM]
-    unsigned int* counters;  // ks > 1: per-tile arrival counts, zero between launches
+    int ks;          // K splits of each split tile (1: no tile is split)
+    int full_units;  // units 0 .. full_units - 1: whole tiles 0 .. full_units - 1
+    int tail0, ntail;  // then tiles tail0 .. tail0 + ntail - 1, each in ks K splits
+    float* ws;       // ks > 1: fp32 partials [ntail * ks][BN][kBM] of the split tiles
+    unsigned int* counters;  // ks > 1: per split tile arrival counts, zero between launches
     const uint16_t* scales;
     const uint16_t* biases;
     uint32_t idesc, tmem_cols;
@@ -138,7 +141,7 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
 // flight together.
 constexpr int kRedU = 4;
 __device__ __forceinline__ void reduce_partials(const TcParams& p, int tile, int n0, int m0, int cols, int et) {
-    const float* base = p.ws + static_cast<int64_t>(tile) * p.ks * p.BN * kBM;
+    const float* base = p.ws + static_cast<int64_t>(tile - p.tail0) * p.ks * p.BN * kBM;
     const int64_t part = static_cast<int64_t>(p.BN) * kBM;  // floats per partial
     const int nchunk = cols * (kBM / 4);
     const bool vec_store = (p.N % 4 == 0) && ((reinterpret_cast<uintptr_t>(p.Y) & 7u) == 0);
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tiles_n = (p.N + kBM - 1) / kBM;
     const int tiles_m = (p.m + p.BN - 1) / p.BN;
     const int num_tiles = tiles_n * tiles_m;
-    const int num_units = num_tiles * p.ks;
+    const int num_units = p.full_units + p.ntail * p.ks;
     const int my_units = blockIdx.x < num_units ? (num_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
     // shared memory: S A tiles | SX activation tiles | kSP packed slots |
@@ -235,15 +238,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto SC_of = [&](int s) { return sb_base + static_cast<uint32_t>(s) * 2u * kStageSB; };
     auto BI_of = [&](int s) { return SC_of(s) + kStageSB; };
     // Work unit t of this CTA: a tile (weight-row tile fastest) and the
-    // k-blocks [kb0, kb1) of its K split.
+    // k-blocks [kb0, kb1) of its K split.  The first full_units units are
+    // whole tiles; the rest are the ks splits of the tiles from tail0 on (the
+    // tiles of a partial last wave, or every tile when there are fewer tiles
+    // than SMs).
+    (void)num_tiles;
     auto unit_of = [&](int t, int& tile, int& split, int& n0, int& m0, int& kb0, int& kb1) {
         const int u = blockIdx.x + t * gridDim.x;
-        tile = u % num_tiles;
-        split = u / num_tiles;
+        if (u < p.full_units) {
+            tile = u;
+            split = -1;  // a whole tile
+            kb0 = 0;
+            kb1 = p.num_kb;
+        } else {
+            const int v = u - p.full_units;
+            tile = p.tail0 + v % p.ntail;
+            split = v / p.ntail;
+            kb0 = static_cast<int>(static_cast<int64_t>(split) * p.num_kb / p.ks);
+            kb1 = static_cast<int>(static_cast<int64_t>(split + 1) * p.num_kb / p.ks);
+        }
         n0 = (tile % tiles_n) * kBM;
         m0 = (tile / tiles_n) * p.BN;
-        kb0 = static_cast<int>(static_cast<int64_t>(split) * p.num_kb / p.ks);
-        kb1 = static_cast<int>(static_cast<int64_t>(split + 1) * p.num_kb / p.ks);
     };
 
     pdl_launch_dependents();
@@ -471,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                (static_cast<uint32_t>(q * 32) << 16);
             const int n = n0 + row;
             const int cols = p.m - m0 < p.BN ? p.m - m0 : p.BN;
-            if (p.ks == 1) {
+            if (split < 0 || p.ks == 1) {
                 for (int c0 = 0; c0 < cols; c0 += 16) {
                     uint32_t r[16];
                     tmem_ld16(d + static_cast<uint32_t>(c0), r);
@@ -495,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // warp's stores are 128 contiguous bytes), free the accumulators,
             // and let the tile's last unit to finish add the ks partials in
             // split order (the same order whichever unit is last).
-            float* part = p.ws + (static_cast<int64_t>(tile) * p.ks + split) * p.BN * kBM;
+            float* part = p.ws + (static_cast<int64_t>(tile - p.tail0) * p.ks + split) * p.BN * kBM;
             for (int c0 = 0; c0 < cols; c0 += 16) {
                 uint32_t r[16];
                 tmem_ld16(d + static_cast<uint32_t>(c0), r);
@@ -510,9 +525,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             __threadfence();  // this thread's partial is visible before the tile's count moves
             named_bar_sync(1, kEpilogueWarps * 32);
             if (ew == 0 && lane == 0) {
-                const unsigned int prev = atomicAdd(p.counters + tile, 1u);
+                const unsigned int prev = atomicAdd(p.counters + (tile - p.tail0), 1u);
                 const bool last = prev == static_cast<unsigned int>(p.ks - 1);
-                if (last) p.counters[tile] = 0u;  // zero again for the next launch
+                if (last) p.counters[tile - p.tail0] = 0u;  // zero again for the next launch
                 *reinterpret_cast<volatile uint32_t*>(last_flag) = last ? 1u : 0u;
             }
             named_bar_sync(1, kEpilogueWarps * 32);
@@ -597,14 +612,38 @@ cudaError_t reset_static_scratch_counters() {
 
 namespace {
 
-// K splits per tile: only when the tiles alone leave SMs idle; as many as
-// keep every split in one wave (units <= SMs) and >= kMinKbPerSplit long.
-int pick_ks(int64_t tiles, int num_kb, int sm_count) {
-    if (tiles >= sm_count) return 1;
-    int64_t ks = sm_count / tiles;
-    const int64_t by_k = num_kb / kMinKbPerSplit;
+// Which tiles split K, and into how many parts.
+//  - Fewer tiles than SMs: every tile splits, into as many parts as keep all
+//    splits in one wave (units <= SMs), each >= kMinKbPerSplit k-blocks.
+//  - Otherwise whole tiles fill the full waves, and the R tiles of a partial
+//    last wave split over the SMs that wave would leave idle (R * ks <= SMs,
+//    each split >= kMinKbPerTail k-blocks): the last wave then takes 1/ks of
+//    a tile's time instead of a whole tile's.
+constexpr int kMinKbPerTail = 4;
+struct SplitPlan {
+    int full_units, tail0, ntail, ks;
+};
+SplitPlan plan_splits(int64_t tiles, int num_kb, int sm_count) {
+    SplitPlan sp{static_cast<int>(tiles), 0, 0, 1};
+    if (tiles < sm_count) {
+        int64_t ks = sm_count / tiles;
+        const int64_t by_k = num_kb / kMinKbPerSplit;
+        if (ks > by_k) ks = by_k;
+        if (ks < 1) ks = 1;
+        sp = SplitPlan{0, 0, static_cast<int>(tiles), static_cast<int>(ks)};
+        return sp;
+    }
+    const int64_t r = tiles % sm_count;
+    if (r == 0) return sp;
+    int64_t ks = sm_count / r;
+    const int64_t by_k = num_kb / kMinKbPerTail;
     if (ks > by_k) ks = by_k;
-    return ks < 1 ? 1 : static_cast<int>(ks);
+    if (ks < 2) return sp;
+    sp.full_units = static_cast<int>(tiles - r);
+    sp.tail0 = static_cast<int>(tiles - r);
+    sp.ntail = static_cast<int>(r);
+    sp.ks = static_cast<int>(ks);
+    return sp;
 }
 
 }  // namespace
@@ -627,9 +666,9 @@ size_t gemm_tc_scratch_bytes(const WeightView& w, int64_t m) {
     const int bn = pick_bn(m);
     const int num_kb = static_cast<int>((w.K + kBK - 1) / kBK);
     const int64_t tiles = ((w.N + kBM - 1) / kBM) * ((m + bn - 1) / bn);
-    const int ks = pick_ks(tiles, num_kb, dev.sm_count);
-    if (ks == 1) return 0;
-    return kCounterBytes + static_cast<size_t>(tiles) * ks * bn * kBM * sizeof(float);
+    const SplitPlan sp = plan_splits(tiles, num_kb, dev.sm_count);
+    if (sp.ks == 1) return 0;
+    return kCounterBytes + static_cast<size_t>(sp.ntail) * sp.ks * bn * kBM * sizeof(float);
 }
 
 cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream,
@@ -648,7 +687,11 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
     p.sb_tma = (w.G % 8 == 0) ? 1 : 0;
     const int64_t tiles = ((w.N + kBM - 1) / kBM) * ((m + p.BN - 1) / p.BN);
     if (tiles > (1ll << 30)) return cudaErrorInvalidValue;
-    p.ks = pick_ks(tiles, p.num_kb, dev.sm_count);
+    const SplitPlan sp = plan_splits(tiles, p.num_kb, dev.sm_count);
+    p.ks = sp.ks;
+    p.full_units = sp.full_units;
+    p.tail0 = sp.tail0;
+    p.ntail = sp.ntail;
     p.scales = w.scales;
     p.biases = w.biases;
     // two A tiles (filled on the SM by the dequant warps), then as many
@@ -684,15 +727,15 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
     static std::atomic<int> configured[64];
     cudaError_t e = ensure_dynamic_smem(k_gemm_tc, smem, configured);
     if (e != cudaSuccess) return e;
-    const int64_t units = tiles * p.ks;
+    const int64_t units = static_cast<int64_t>(p.full_units) + static_cast<int64_t>(p.ntail) * p.ks;
     const int grid = static_cast<int>(units < dev.sm_count ? units : dev.sm_count);
     if (p.ks == 1) {
         e = launch_pdl(k_gemm_tc, dim3(grid), dim3(kThreads), smem, stream, tm_x, wm.packed, wm.scales, wm.biases, p);
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
-    const size_t part_bytes = static_cast<size_t>(units) * p.BN * kBM * sizeof(float);
-    if (tiles * sizeof(unsigned int) > kCounterBytes) return cudaErrorInvalidValue;
+    const size_t part_bytes = static_cast<size_t>(p.ntail) * p.ks * p.BN * kBM * sizeof(float);
+    if (static_cast<size_t>(p.ntail) * sizeof(unsigned int) > kCounterBytes) return cudaErrorInvalidValue;
     if (scratch == TC_SCRATCH_STATIC) {
         // the library's static buffer: counters already zero, nothing allocated
         if (kCounterBytes + part_bytes > kStaticScratchBytes) return cudaErrorMemoryAllocation;
@@ -707,7 +750,7 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
     }
     // K split: the fp32 partials and the per-tile counters come from the
     // library's stream-ordered pool, allocated and freed in order on the stream
-    const size_t bytes = part_bytes + static_cast<size_t>(tiles) * sizeof(unsigned int);
+    const size_t bytes = part_bytes + static_cast<size_t>(p.ntail) * sizeof(unsigned int);
     cudaMemPool_t pool;
     e = workspace_pool(dev.device, &pool);
     if (e != cudaSuccess) return e;
@@ -716,7 +759,7 @@ cudaError_t launch_gemm_tc(const WeightView& w, const void* X, void* Y, int64_t 
     if (e != cudaSuccess) return e;
     p.ws = static_cast<float*>(ws);
     p.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + part_bytes);
-    e = cudaMemsetAsync(p.counters, 0, static_cast<size_t>(tiles) * sizeof(unsigned int), stream);
+    e = cudaMemsetAsync(p.counters, 0, static_cast<size_t>(p.ntail) * sizeof(unsigned int), stream);
     if (e == cudaSuccess)
         e = launch_pdl(k_gemm_tc, dim3(grid), dim3(kThreads), smem, stream, tm_x, wm.packed, wm.scales, wm.biases, p);
     if (e == cudaSuccess) e = cudaGetLastError();
