@@ -189,9 +189,13 @@ enum {
                                   when group_size % 16 == 0; any m, in passes of up to
                                   8 rows, for other group sizes with group_size % 4 == 0
                                   and in_features % 16 == 0 */
-    MLXQ_GEMM_SMALLM_GROUPS = 5 /* weight-streaming kernel on the tensor pipe, m <= 32:
+    MLXQ_GEMM_SMALLM_GROUPS = 5, /* weight-streaming kernel on the tensor pipe, m <= 32:
                                   each SM walks a balanced range of 16-row tiles in
                                   groups; in_features % 128 == 0, group_size 16/32/64 */
+    MLXQ_GEMM_SMALLM_TC = 6    /* weight-streaming kernel on tcgen05, m <= 64: the
+                                  dequantised weight is the M = 128 operand, the
+                                  activations the N operand; in_features % 128 == 0,
+                                  group_size 16/32/64/128, (in/group_size) % 8 == 0 */
 };
 
 /* mlxq_gemm with an explicit kernel; MLXQ_ERR_UNSUPPORTED if that kernel

@@ -468,6 +468,23 @@ def test_gemm_smallm_tile_groups(N, K, gs, m):
     assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_SMALLM_GROUPS), ref, f"smallm-groups m={m} {N}x{K}")
 
 
+# the tcgen05 small-m kernel: K % 128 == 0, gs 16..128 with (K/gs) % 8 == 0;
+# several tile groups per CTA, partial last groups, a ragged last tile
+TCSM_SHAPES = [(512, 1024, 64), (300, 4096, 32), (77, 512, 16), (5000, 1152, 16), (2100, 2304, 32),
+               (14336 + 8, 512, 64), (256, 14336, 128), (40000 + 3, 1024, 128)]
+
+
+@pytest.mark.parametrize("N,K,gs", TCSM_SHAPES)
+@pytest.mark.parametrize("m", [1, 9, 16, 17, 32, 33, 64])
+def test_gemm_smallm_tcgen05(N, K, gs, m):
+    W, g = make(13, N, K, gs)
+    X = synth.activations(g, m, K)
+    ref = oracle.gemm(*W.host, gs, X)
+    assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_SMALLM_TC), ref, f"smallm-tc m={m} {N}x{K}")
+    if m > 32:
+        assert_close(run_gemm(W, X, m, mq.MLXQ_GEMM_AUTO), ref, f"auto m={m} {N}x{K}")
+
+
 def test_gemm_smallm_tile_groups_refuses_what_it_cannot_take():
     W, g = make(12, 256, 14336, 128)  # gs = 128: not taken
     X = dev(synth.activations(g, 4, 14336))

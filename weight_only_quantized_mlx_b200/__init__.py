@@ -36,6 +36,7 @@ MLXQ_GEMM_SMALLM = 2
 MLXQ_GEMM_TCGEN05 = 3
 MLXQ_GEMM_SMALLM_FFMA = 4
 MLXQ_GEMM_SMALLM_GROUPS = 5
+MLXQ_GEMM_SMALLM_TC = 6
 
 MLXQ_WEIGHT_STATIC = 1
 

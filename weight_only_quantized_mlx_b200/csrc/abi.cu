@@ -598,7 +598,7 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
     WeightView v;
     int rc = check_weight(w, v);
     if (rc) return rc;
-    if (kernel < MLXQ_GEMM_AUTO || kernel > MLXQ_GEMM_SMALLM_GROUPS)
+    if (kernel < MLXQ_GEMM_AUTO || kernel > MLXQ_GEMM_SMALLM_TC)
         return fail(MLXQ_ERR_INVALID_ARG, "unknown gemm kernel id %d", kernel);
     if (m == 0) return ok();
     const int64_t M = m;
@@ -614,6 +614,7 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
     int k = kernel;
     if (k == MLXQ_GEMM_AUTO) {
         if (M == 1) k = MLXQ_GEMM_ROWS;
+        else if (smallm_tc_preferred(v, M, x)) k = MLXQ_GEMM_SMALLM_TC;
         else if (M <= kStreamMmaMaxM && smallm_preferred(v, M, x)) k = MLXQ_GEMM_SMALLM_GROUPS;
         else if (M <= kStreamMmaMaxM && stream_mma_supported(v, GEMV_PLAIN, M, x, nullptr, nullptr))
             k = MLXQ_GEMM_SMALLM;
@@ -633,6 +634,11 @@ int gemm_impl(const mlxq_weight* w, const void* x, void* y, uint32_t m, int kern
             }
             return ok();
         }
+        case MLXQ_GEMM_SMALLM_TC:
+            if (!smallm_tc_supported(v, M, x))
+                return fail(MLXQ_ERR_UNSUPPORTED, "small-m tcgen05 kernel cannot take m=%lld, K=%lld, group_size=%lld",
+                            static_cast<long long>(M), static_cast<long long>(v.K), static_cast<long long>(v.gs));
+            return launch_status(launch_smallm_tc(v, x, y, M, s), "small-m tcgen05 gemm launch");
         case MLXQ_GEMM_SMALLM_GROUPS:
             if (!smallm_supported(v, M, x))
                 return fail(MLXQ_ERR_UNSUPPORTED, "small-m tile-group kernel cannot take m=%lld, K=%lld, group_size=%lld",

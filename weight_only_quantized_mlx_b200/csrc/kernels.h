@@ -98,6 +98,10 @@ cudaError_t launch_stream_mma(const WeightView& w, int mode, int64_t m, const vo
 // Small-m gemm, 1 <= m <= 32, weight tiles walked in groups by one CTA per
 // SM (tensor-pipe fragments, activations copied with each stage).
 bool smallm_supported(const WeightView& w, int64_t m, const void* X);
+// Small m on tcgen05 (swap-AB: weights as the M = 128 operand), 1 <= m <= 64.
+bool smallm_tc_supported(const WeightView& w, int64_t m, const void* X);
+bool smallm_tc_preferred(const WeightView& w, int64_t m, const void* X);
+cudaError_t launch_smallm_tc(const WeightView& w, const void* X, void* Y, int64_t m, cudaStream_t stream);
 // supported, and measured faster than the per-row-pair streaming kernel:
 // 8 < m and at least 6 tiles of 16 rows per SM
 bool smallm_preferred(const WeightView& w, int64_t m, const void* X);
