@@ -11,15 +11,17 @@
 // groups of up to 8 tiles (128 rows).  Each group streams K in 128-code
 // stages:
 //   warp 0      TMA: per stage one box of the group's codes ([rows x 128
-//               bytes], 128-byte swizzle) and one 3-D box of the stage's
-//               activation columns ([2 k-blocks][BN rows][64 columns],
-//               128-byte swizzle, zero past m and K); per 16 scale groups one
-//               [rows x 16] box each of scales and biases
-//   warp 1      allocates TMEM (two fp32 accumulators of BN columns) and,
-//               from one lane, issues tcgen05.mma kind::f16 (BF16 x BF16 ->
-//               fp32): 8 per stage, A from the stage's A tile, B from the
-//               stage's activation box
-//   warps 2-17  dequantise the stage's codes into the A tile (K-major,
+//               bytes], 128-byte swizzle) into the code ring; per 16 scale
+//               groups one [rows x 16] box each of scales and biases
+//   warp 2      TMA: per stage one 3-D box of the activation columns ([2
+//               k-blocks][BN rows][64 columns], 128-byte swizzle, zero past m
+//               and K) into its own ring, so a code slot is free again as soon
+//               as the codes are dequantised, not when the MMAs are done
+//   warp 1      allocates TMEM (one fp32 accumulator of BN columns) and, from
+//               one lane, issues tcgen05.mma kind::f16 (BF16 x BF16 -> fp32):
+//               8 per stage, A from the stage's A tile, B from its activation
+//               box
+//   warps 3-18  dequantise the stage's codes into the A tile (K-major,
 //               128-byte swizzle: the BF16 weight dequantize_to writes), and
 //               at the end of a group read the accumulator (tcgen05.ld) and
 //               store the group's outputs
@@ -37,9 +39,10 @@ namespace mlxq {
 namespace {
 
 constexpr int kStW = 16;             // dequantising warps
-constexpr int kStThreads = (kStW + 2) * 32;
+constexpr int kStThreads = (kStW + 3) * 32;
 constexpr int kStKB = 128;           // codes per stage (two 64-code k-blocks)
-constexpr int kStMaxS = 6;           // stage ring depth
+constexpr int kStMaxS = 8;           // code ring depth
+constexpr int kStMaxX = 4;           // activation ring depth
 constexpr int kStTabGroups = 16;     // scale groups per table box
 constexpr uint32_t kStA = 128u * 128u;  // one k-block's A tile: 128 rows x 128 bytes
 constexpr int kStMaxGP = 8;          // tiles per group
@@ -51,13 +54,12 @@ struct StParams {
     int P;              // 16-row tiles
     int gp;             // tiles per group (<= 8)
     int num_kb;         // stages per group pass
-    int S;              // stage ring depth
+    int S, SX;          // code ring depth, activation ring depth
     int tab_every;      // stages per table box (16 * gs / 128)
-    uint32_t code_bytes;   // codes box of a stage: gp * 16 rows x 128 bytes
-    uint32_t x_bytes;      // activation box of a stage: 2 x BN x 128 bytes
-    uint32_t stage_bytes;  // code_bytes + x_bytes, 1024-byte multiple
+    uint32_t code_bytes;   // codes box of a stage: gp * 16 rows x 128 bytes (1024-byte multiple)
+    uint32_t x_bytes;      // activation box of a stage: 2 x BN x 128 bytes (1024-byte multiple)
     uint32_t tab_bytes;    // one table box: gp * 16 rows x 32 bytes
-    uint32_t a_off, t_off, bar_off;  // from the 1024-aligned shared-memory base
+    uint32_t x_off, a_off, t_off, bar_off;  // from the 1024-aligned shared-memory base
     uint32_t idesc;
     unsigned int* status;
 };
@@ -123,13 +125,15 @@ __global__ void __launch_bounds__(kStThreads, 1) k_smallm_tc(const __grid_consta
     uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int S = p.S;
+    const int S = p.S, SX = p.SX;
     const int t0 = static_cast<int>(static_cast<int64_t>(p.P) * blockIdx.x / gridDim.x);
     const int t1 = static_cast<int>(static_cast<int64_t>(p.P) * (blockIdx.x + 1) / gridDim.x);
     const int ngroups = (t1 - t0 + p.gp - 1) / p.gp;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);  // stage landed (TMA)
-    uint64_t* sempty = full + kStMaxS;   // stage free: codes read (16 warps) and MMAs done (commit)
-    uint64_t* tfull = sempty + kStMaxS;  // table box landed
+    uint64_t* cfull = reinterpret_cast<uint64_t*>(smem + p.bar_off);  // codes landed (TMA)
+    uint64_t* cempty = cfull + kStMaxS;  // codes read (16 warps)
+    uint64_t* xfull = cempty + kStMaxS;  // activation box landed (TMA)
+    uint64_t* xempty = xfull + kStMaxX;  // activation box read by the MMAs (commit)
+    uint64_t* tfull = xempty + kStMaxX;  // table box landed
     uint64_t* tempty = tfull + 2;        // table box read
     uint64_t* afull = tempty + 2;        // A tile written (16 warps)
     uint64_t* aempty = afull + kStNA;    // A tile read by the MMAs (commit)
@@ -137,7 +141,8 @@ __global__ void __launch_bounds__(kStThreads, 1) k_smallm_tc(const __grid_consta
     uint64_t* dempty = dfull + 1;        // the accumulator read out (16 warps)
     uint64_t* drain = dempty + 1;        // the MMA thread's last commit
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-    auto stage_of = [&](int s) { return sbase + static_cast<uint32_t>(s) * p.stage_bytes; };
+    auto codes_of = [&](int s) { return sbase + static_cast<uint32_t>(s) * p.code_bytes; };
+    auto x_of = [&](int s) { return sbase + p.x_off + static_cast<uint32_t>(s) * p.x_bytes; };
     auto a_of = [&](int a) { return sbase + p.a_off + static_cast<uint32_t>(a) * 2u * kStA; };
     auto tab_of = [&](int t) { return sbase + p.t_off + static_cast<uint32_t>(t) * 2u * p.tab_bytes; };
     constexpr uint32_t kTmemCols = BN < 32 ? 32u : static_cast<uint32_t>(BN);
@@ -145,8 +150,12 @@ __global__ void __launch_bounds__(kStThreads, 1) k_smallm_tc(const __grid_consta
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_u32(&full[s]), 1);
-            mbar_init(smem_u32(&sempty[s]), kStW + 1);
+            mbar_init(smem_u32(&cfull[s]), 1);
+            mbar_init(smem_u32(&cempty[s]), kStW);
+        }
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(smem_u32(&xfull[s]), 1);
+            mbar_init(smem_u32(&xempty[s]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&tfull[i]), 1);
@@ -172,14 +181,12 @@ __global__ void __launch_bounds__(kStThreads, 1) k_smallm_tc(const __grid_consta
     pdl_wait();  // activations, weights and Y belong to earlier work
 
     if (warp == 0) {
-        // ---------------- producer ----------------
+        // ---------------- codes and tables producer ----------------
         if (lane == 0) {
             prefetch_tmap(&maps.codes[p.gp - 1]);
             prefetch_tmap(&maps.sc[p.gp - 1]);
             prefetch_tmap(&maps.bi[p.gp - 1]);
-            prefetch_tmap(&maps.x);
             const uint64_t pol = policy_evict_first();
-            const uint64_t pol_x = policy_evict_last();  // every CTA reads the same activations
             bool ok = true;
             int it = 0, ti = 0;
             for (int grp = 0; grp < ngroups && ok; ++grp) {
@@ -198,20 +205,40 @@ __global__ void __launch_bounds__(kStThreads, 1) k_smallm_tc(const __grid_consta
                         ++ti;
                     }
                     const int s = it % S;
-                    if (it >= S) ok = mbar_wait(smem_u32(&sempty[s]), ((it / S) - 1) & 1, p.status);
+                    if (it >= S) ok = mbar_wait(smem_u32(&cempty[s]), ((it / S) - 1) & 1, p.status);
                     if (!ok) break;
-                    const uint32_t fb = smem_u32(&full[s]);
-                    mbar_arrive_expect_tx(fb, static_cast<uint32_t>(nt) * 16u * 128u + p.x_bytes);
-                    tma_load_2d(stage_of(s), &maps.codes[nt - 1], kb * kStKB, ta * 16, fb, pol);
-                    tma_load_3d(stage_of(s) + p.code_bytes, &maps.x, 0, 0, kb * 2, fb, pol_x);
+                    const uint32_t fb = smem_u32(&cfull[s]);
+                    mbar_arrive_expect_tx(fb, static_cast<uint32_t>(nt) * 16u * 128u);
+                    tma_load_2d(codes_of(s), &maps.codes[nt - 1], kb * kStKB, ta * 16, fb, pol);
                     ++it;
                 }
             }
             // every issued copy has landed before the CTA may exit
             for (int u = it > S ? it - S : 0; u < it; ++u)
-                if (!mbar_wait(smem_u32(&full[u % S]), (u / S) & 1, p.status)) break;
+                if (!mbar_wait(smem_u32(&cfull[u % S]), (u / S) & 1, p.status)) break;
             for (int u = ti > 2 ? ti - 2 : 0; u < ti; ++u)
                 if (!mbar_wait(smem_u32(&tfull[u % 2]), (u / 2) & 1, p.status)) break;
+        }
+    } else if (warp == 2) {
+        // ---------------- activation producer ----------------
+        if (lane == 0) {
+            prefetch_tmap(&maps.x);
+            const uint64_t pol_x = policy_evict_last();  // every CTA reads the same activations
+            bool ok = true;
+            int it = 0;
+            for (int grp = 0; grp < ngroups && ok; ++grp) {
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    const int s = it % SX;
+                    if (it >= SX) ok = mbar_wait(smem_u32(&xempty[s]), ((it / SX) - 1) & 1, p.status);
+                    if (!ok) break;
+                    const uint32_t fb = smem_u32(&xfull[s]);
+                    mbar_arrive_expect_tx(fb, p.x_bytes);
+                    tma_load_3d(x_of(s), &maps.x, 0, 0, kb * 2, fb, pol_x);
+                    ++it;
+                }
+            }
+            for (int u = it > SX ? it - SX : 0; u < it; ++u)
+                if (!mbar_wait(smem_u32(&xfull[u % SX]), (u / SX) & 1, p.status)) break;
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -224,21 +251,21 @@ __global__ void __launch_bounds__(kStThreads, 1) k_smallm_tc(const __grid_consta
                 if (!ok) break;
                 st_fence_after();
                 for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-                    const int s = it % S, a = it % kStNA;
+                    const int sx = it % SX, a = it % kStNA;
                     ok = mbar_wait(smem_u32(&afull[a]), (it / kStNA) & 1, p.status);
-                    if (ok) ok = mbar_wait(smem_u32(&full[s]), (it / S) & 1, p.status);
+                    if (ok) ok = mbar_wait(smem_u32(&xfull[sx]), (it / SX) & 1, p.status);
                     if (!ok) break;  // operands not there: issue nothing more
                     st_fence_after();
 #pragma unroll
                     for (int kbi = 0; kbi < 2; ++kbi) {
                         const uint64_t ad = st_desc(a_of(a) + static_cast<uint32_t>(kbi) * kStA);
-                        const uint64_t bd = st_desc(stage_of(s) + p.code_bytes + static_cast<uint32_t>(kbi * BN) * 128u);
+                        const uint64_t bd = st_desc(x_of(sx) + static_cast<uint32_t>(kbi * BN) * 128u);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)  // 16 BF16 (32 bytes) along K per MMA
                             st_mma(tmem_base, ad + 2u * kk, bd + 2u * kk, p.idesc, (kb | kbi | kk) != 0 ? 1u : 0u);
                     }
                     st_commit(smem_u32(&aempty[a]));
-                    st_commit(smem_u32(&sempty[s]));
+                    st_commit(smem_u32(&xempty[sx]));
                 }
                 if (ok) st_commit(smem_u32(dfull));
             }
@@ -249,7 +276,7 @@ __global__ void __launch_bounds__(kStThreads, 1) k_smallm_tc(const __grid_consta
         __syncwarp();
     } else {
         // ---------------- dequantising warps; then each group's outputs ----------------
-        const int dw = warp - 2;        // 0 .. 15
+        const int dw = warp - 3;        // 0 .. 15
         const int dt = dw * 32 + lane;  // 0 .. 511
         const float2 m2 = make_float2(-kMagic, -kMagic);
         bool ok = true;
@@ -258,21 +285,46 @@ __global__ void __launch_bounds__(kStThreads, 1) k_smallm_tc(const __grid_consta
             const int ta = t0 + grp * p.gp;
             const int nt = min(p.gp, t1 - ta);
             const int units = nt * 16 * 8;  // (row, 16-code chunk) pairs of a stage
+            // This thread's units (at most two), the same in every stage of the
+            // group.  16 consecutive units cover rows 2b and 2b + 1; each 8-lane
+            // phase takes four chunks of one row and the other four of the other
+            // row, so its code loads and its A stores each hit 8 distinct 16-byte
+            // bank groups.
+            uint32_t ld_off[2], st0[2], st1[2], trow[2];
+            int cch[2];
+            bool has[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int u = dt + i * kStW * 32;
+                has[i] = u < units;
+                const int q = u & 15, tq = (q >> 2) & 1;
+                const int r = 2 * (u >> 4) + (tq ^ (q >> 3));
+                const int c = (q & 3) + 4 * tq;
+                const uint32_t sw = static_cast<uint32_t>(r & 7);
+                ld_off[i] = static_cast<uint32_t>(r) * 128u + ((static_cast<uint32_t>(c) ^ sw) << 4);
+                // chunk c lands in k-block c / 4 of the A tile, 16-byte units
+                // 2 (c % 4) and 2 (c % 4) + 1 of row r, placed by the swizzle
+                const uint32_t arow = static_cast<uint32_t>(c >> 2) * kStA + static_cast<uint32_t>(r) * 128u;
+                st0[i] = arow + (((2u * static_cast<uint32_t>(c & 3)) ^ sw) << 4);
+                st1[i] = arow + (((2u * static_cast<uint32_t>(c & 3) + 1u) ^ sw) << 4);
+                trow[i] = static_cast<uint32_t>(r * kStTabGroups) * 2u;
+                cch[i] = c;
+            }
             for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
                 const int ts = ti % 2;
                 if (kb % kTabEvery == 0 && ok) ok = mbar_wait(smem_u32(&tfull[ts]), (ti / 2) & 1, p.status);
                 const int s = it % S, a = it % kStNA;
-                if (ok) ok = mbar_wait(smem_u32(&full[s]), (it / S) & 1, p.status);
+                if (ok) ok = mbar_wait(smem_u32(&cfull[s]), (it / S) & 1, p.status);
                 // the MMAs that last read this A tile are done
                 if (it >= kStNA && ok) ok = mbar_wait(smem_u32(&aempty[a]), ((it / kStNA) - 1) & 1, p.status);
-                const uint32_t st = stage_of(s);
+                const uint32_t cs = codes_of(s), as = a_of(a);
                 const uint32_t sca = tab_of(ts), bia = sca + p.tab_bytes;
                 const int gbase = (kb % kTabEvery) * kStKB;  // codes of the table box before this stage
-                for (int u = dt; u < units; u += kStW * 32) {
-                    const int r = u >> 3, c = u & 7;
-                    const uint32_t sw = static_cast<uint32_t>(r & 7);
-                    const uint4 wq = lds128(st + static_cast<uint32_t>(r) * 128u + ((static_cast<uint32_t>(c) ^ sw) << 4));
-                    const uint32_t so = static_cast<uint32_t>(r * kStTabGroups + (gbase + 16 * c) / GS) * 2u;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (!has[i]) continue;
+                    const uint4 wq = lds128(cs + ld_off[i]);
+                    const uint32_t so = trow[i] + static_cast<uint32_t>((gbase + 16 * cch[i]) / GS) * 2u;
                     const float sv = bf16_bits_to_f32(lds16(sca + so)), bv = bf16_bits_to_f32(lds16(bia + so));
                     const float2 s2 = make_float2(sv, sv), b2 = make_float2(bv, bv);
                     const uint32_t words[4] = {wq.x, wq.y, wq.z, wq.w};
@@ -287,18 +339,14 @@ __global__ void __launch_bounds__(kStThreads, 1) k_smallm_tc(const __grid_consta
                         o[2 * j] = pack_bf16x2(w01.x, w01.y);
                         o[2 * j + 1] = pack_bf16x2(w23.x, w23.y);
                     }
-                    // chunk c lands in k-block c / 4 of the A tile, 16-byte units
-                    // 2 (c % 4) and 2 (c % 4) + 1 of row r, placed by the swizzle
-                    const uint32_t arow = a_of(a) + static_cast<uint32_t>(c >> 2) * kStA + static_cast<uint32_t>(r) * 128u;
-                    const uint32_t cc = static_cast<uint32_t>(c & 3);
-                    st_sts128(arow + (((2u * cc) ^ sw) << 4), o[0], o[1], o[2], o[3]);
-                    st_sts128(arow + (((2u * cc + 1u) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+                    st_sts128(as + st0[i], o[0], o[1], o[2], o[3]);
+                    st_sts128(as + st1[i], o[4], o[5], o[6], o[7]);
                 }
                 fence_proxy_async_smem();  // the tensor core reads the A tile through the async proxy
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(smem_u32(&afull[a]));
-                    mbar_arrive(smem_u32(&sempty[s]));  // this warp is done with the stage's codes
+                    mbar_arrive(smem_u32(&cempty[s]));  // this warp is done with the stage's codes
                 }
                 if (kb % kTabEvery == kTabEvery - 1 || kb == p.num_kb - 1) {
                     if (lane == 0) mbar_arrive(smem_u32(&tempty[ts]));
@@ -349,7 +397,7 @@ struct StPlan {
     size_t smem;
 };
 
-constexpr size_t kStBarBytes = 256;
+constexpr size_t kStBarBytes = 512;
 
 bool plan_st(const WeightView& w, int64_t m, StPlan& pl) {
     const DeviceInfo& dev = device_info();
@@ -373,16 +421,17 @@ bool plan_st(const WeightView& w, int64_t m, StPlan& pl) {
     p.tab_every = kStTabGroups * p.gs / kStKB;
     p.code_bytes = static_cast<uint32_t>(p.gp) * 16u * 128u;
     p.x_bytes = 2u * static_cast<uint32_t>(pl.bn) * 128u;
-    p.stage_bytes = (p.code_bytes + p.x_bytes + 1023u) / 1024u * 1024u;
     p.tab_bytes = static_cast<uint32_t>(p.gp) * 16u * 2u * kStTabGroups;
     const size_t a_bytes = static_cast<size_t>(kStNA) * 2 * kStA;
     const size_t fixed = 1024 + a_bytes + 4 * static_cast<size_t>(p.tab_bytes) + kStBarBytes;
     const size_t budget = static_cast<size_t>(dev.max_smem_optin);
-    if (budget < fixed + 2 * static_cast<size_t>(p.stage_bytes)) return false;
-    int S = static_cast<int>((budget - fixed) / p.stage_bytes);
+    p.SX = kStMaxX;
+    if (budget < fixed + static_cast<size_t>(p.SX) * p.x_bytes + 2 * static_cast<size_t>(p.code_bytes)) return false;
+    int S = static_cast<int>((budget - fixed - static_cast<size_t>(p.SX) * p.x_bytes) / p.code_bytes);
     if (S > kStMaxS) S = kStMaxS;
     p.S = S;
-    p.a_off = static_cast<uint32_t>(S) * p.stage_bytes;
+    p.x_off = static_cast<uint32_t>(S) * p.code_bytes;
+    p.a_off = p.x_off + static_cast<uint32_t>(p.SX) * p.x_bytes;
     p.t_off = p.a_off + static_cast<uint32_t>(a_bytes);
     p.bar_off = p.t_off + 4u * p.tab_bytes;
     pl.smem = 1024 + p.bar_off + kStBarBytes;
