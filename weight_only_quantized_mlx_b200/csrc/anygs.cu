@@ -12,9 +12,9 @@
 //
 //   k_anygs_gemv    y = W h (+ resid) with h = x rows (MT of them per pass)
 //                   or silu(gate) * up; each warp takes two weight rows at a
-//                   time, lanes split K, the activations sit in shared
-//                   memory, and the weight element is the BF16 value
-//                   dequantize_to writes
+//                   time (paired in fp32x2 operations), lanes split K, the
+//                   activations sit in shared memory, and the weight element
+//                   is the BF16 value dequantize_to writes
 //   k_dequant_anygs dequantize_to: one 16-code chunk per thread per step, 32
 //                   (or 2 x 16) bytes stored
 #include <atomic>
@@ -53,11 +53,14 @@ __device__ __forceinline__ int word_group_step(int r, int j, int gs) {
     return (t >= gs) + (t >= 2 * gs) + (t >= 3 * gs);
 }
 
-// BF16-rounded weight of code c (byte J of word w), as fp32
+// The BF16-rounded weights of byte J of word u (row r0) and of word v (row
+// r1), as an fp32 pair: paired subtract and fma, one two-value pack.
 template <int J>
-__device__ __forceinline__ float weight_of(uint32_t w, float s, float b) {
-    const float q = code_magic<J>(w) - kMagic;
-    return bf16_bits_to_f32(__bfloat16_as_ushort(__float2bfloat16_rn(__fmaf_rn(s, q, b))));
+__device__ __forceinline__ float2 weight_pair(uint32_t u, uint32_t v, float2 s2, float2 b2) {
+    const float2 q = __fadd2_rn(make_float2(code_magic<J>(u), code_magic<J>(v)), make_float2(-kMagic, -kMagic));
+    const float2 f = __ffma2_rn(q, s2, b2);
+    const uint32_t w = pack_bf16x2(f.x, f.y);
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
 // MT: activation rows per pass (plain mode); 1 for the silu modes.
@@ -126,9 +129,9 @@ __global__ void __launch_bounds__(kAgThreads) k_anygs_gemv(const AgParams p) {
         const uint16_t* s1 = p.scales + r1 * p.G;
         const uint16_t* b0 = p.biases + r0 * p.G;
         const uint16_t* b1 = p.biases + r1 * p.G;
-        float acc0[MT], acc1[MT];
+        float2 acc[MT];  // (row r0, row r1)
 #pragma unroll
-        for (int i = 0; i < MT; ++i) acc0[i] = acc1[i] = 0.f;
+        for (int i = 0; i < MT; ++i) acc[i] = make_float2(0.f, 0.f);
         // the lane's first chunk starts at code 16 * lane
         int g = (16 * lane) / p.gs;
         int r = 16 * lane - g * p.gs;
@@ -169,15 +172,14 @@ __global__ void __launch_bounds__(kAgThreads) k_anygs_gemv(const AgParams p) {
                     const uint32_t a1[4] = {q1[u].x, q1[u].y, q1[u].z, q1[u].w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        float v0[4], v1[4];
-                        v0[0] = weight_of<0>(a0[j], sc0[u][j], bi0[u][j]);
-                        v0[1] = weight_of<1>(a0[j], sc0[u][j], bi0[u][j]);
-                        v0[2] = weight_of<2>(a0[j], sc0[u][j], bi0[u][j]);
-                        v0[3] = weight_of<3>(a0[j], sc0[u][j], bi0[u][j]);
-                        v1[0] = weight_of<0>(a1[j], sc1[u][j], bi1[u][j]);
-                        v1[1] = weight_of<1>(a1[j], sc1[u][j], bi1[u][j]);
-                        v1[2] = weight_of<2>(a1[j], sc1[u][j], bi1[u][j]);
-                        v1[3] = weight_of<3>(a1[j], sc1[u][j], bi1[u][j]);
+                        // the two rows side by side in paired fp32 operations
+                        const float2 s2 = make_float2(sc0[u][j], sc1[u][j]);
+                        const float2 b2 = make_float2(bi0[u][j], bi1[u][j]);
+                        float2 v[4];
+                        v[0] = weight_pair<0>(a0[j], a1[j], s2, b2);
+                        v[1] = weight_pair<1>(a0[j], a1[j], s2, b2);
+                        v[2] = weight_pair<2>(a0[j], a1[j], s2, b2);
+                        v[3] = weight_pair<3>(a0[j], a1[j], s2, b2);
                         const int k = 16 * c + 4 * j;
                         if (MODE == GEMV_PLAIN) {
                             const uint16_t* xs = reinterpret_cast<const uint16_t*>(smem_ag);
@@ -186,31 +188,29 @@ __global__ void __launch_bounds__(kAgThreads) k_anygs_gemv(const AgParams p) {
                                 const uint2 xv = *reinterpret_cast<const uint2*>(xs + i * K + k);
                                 const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xFFFF0000u);
                                 const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xFFFF0000u);
-                                acc0[i] = __fmaf_rn(v0[0], x0, acc0[i]);
-                                acc1[i] = __fmaf_rn(v1[0], x0, acc1[i]);
-                                acc0[i] = __fmaf_rn(v0[1], x1, acc0[i]);
-                                acc1[i] = __fmaf_rn(v1[1], x1, acc1[i]);
-                                acc0[i] = __fmaf_rn(v0[2], x2, acc0[i]);
-                                acc1[i] = __fmaf_rn(v1[2], x2, acc1[i]);
-                                acc0[i] = __fmaf_rn(v0[3], x3, acc0[i]);
-                                acc1[i] = __fmaf_rn(v1[3], x3, acc1[i]);
+                                acc[i] = __ffma2_rn(v[0], make_float2(x0, x0), acc[i]);
+                                acc[i] = __ffma2_rn(v[1], make_float2(x1, x1), acc[i]);
+                                acc[i] = __ffma2_rn(v[2], make_float2(x2, x2), acc[i]);
+                                acc[i] = __ffma2_rn(v[3], make_float2(x3, x3), acc[i]);
                             }
                         } else {
                             const float4 h = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(smem_ag) + k);
-                            acc0[0] = __fmaf_rn(v0[0], h.x, acc0[0]);
-                            acc1[0] = __fmaf_rn(v1[0], h.x, acc1[0]);
-                            acc0[0] = __fmaf_rn(v0[1], h.y, acc0[0]);
-                            acc1[0] = __fmaf_rn(v1[1], h.y, acc1[0]);
-                            acc0[0] = __fmaf_rn(v0[2], h.z, acc0[0]);
-                            acc1[0] = __fmaf_rn(v1[2], h.z, acc1[0]);
-                            acc0[0] = __fmaf_rn(v0[3], h.w, acc0[0]);
-                            acc1[0] = __fmaf_rn(v1[3], h.w, acc1[0]);
+                            acc[0] = __ffma2_rn(v[0], make_float2(h.x, h.x), acc[0]);
+                            acc[0] = __ffma2_rn(v[1], make_float2(h.y, h.y), acc[0]);
+                            acc[0] = __ffma2_rn(v[2], make_float2(h.z, h.z), acc[0]);
+                            acc[0] = __ffma2_rn(v[3], make_float2(h.w, h.w), acc[0]);
                         }
                     }
                 }
             }
         }
         // the lanes' partial sums, in a fixed butterfly order
+        float acc0[MT], acc1[MT];
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+            acc0[i] = acc[i].x;
+            acc1[i] = acc[i].y;
+        }
 #pragma unroll
         for (int i = 0; i < MT; ++i) {
 #pragma unroll
