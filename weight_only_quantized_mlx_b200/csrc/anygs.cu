@@ -27,7 +27,10 @@ namespace {
 
 constexpr int kAgWarps = 8;
 constexpr int kAgThreads = kAgWarps * 32;
-constexpr int kAgUnroll = 2;  // chunks per lane whose loads are issued together
+// chunks per lane whose loads are issued together: 4 with one activation row
+// per pass, 2 with more (registers)
+template <int MT>
+constexpr int ag_unroll() { return MT == 1 ? 4 : 2; }
 
 struct AgParams {
     const uint8_t* packed;   // [N, K] codes, 16-byte aligned rows
@@ -66,6 +69,7 @@ __device__ __forceinline__ float2 weight_pair(uint32_t u, uint32_t v, float2 s2,
 // MT: activation rows per pass (plain mode); 1 for the silu modes.
 template <int MODE, int MT>
 __global__ void __launch_bounds__(kAgThreads) k_anygs_gemv(const AgParams p) {
+    constexpr int kAgUnroll = ag_unroll<MT>();
     extern __shared__ __align__(16) uint8_t smem_ag[];
     const int lane = threadIdx.x & 31;
     const int K = p.K;
