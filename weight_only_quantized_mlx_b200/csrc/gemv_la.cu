@@ -21,6 +21,8 @@
 // All waits are bounded.  After a wait gives up, the producer stops issuing
 // copies and, before the CTA exits, waits (bounded) for the copies it has in
 // flight, so no copy lands in shared memory the CTA no longer owns.
+#include <cstring>
+
 #include "device_common.cuh"
 #include "kernels.h"
 #include "tensor_map.h"
@@ -45,7 +47,10 @@ struct LaParams {
     int Kpad;                // num_kb * stage width (activation staging, zero past K)
     int pf_stages;           // stages prefetched to L2 before the dependency wait
     int pre_wait;            // stages copied into shared memory before it (static weights; <= S)
-    uint32_t box_bytes;      // npair * 16 rows * 128 bytes
+    uint32_t box_rows;       // rows of one 128-code column in shared memory (R, or npair * 16)
+    uint32_t box_bytes;      // box_rows * 128 bytes
+    int codes3;              // > 0: 3-D copies of this many 128-code columns each
+    uint32_t tab_off;        // tables within a stage: after the columns and the rows a tile reads past R
     uint32_t sb_bytes;       // one table (scales or biases) of a stage, 128-byte padded
     uint32_t stage_bytes;    // 1024-byte multiple
     uint32_t xs_off, red_off, bar_off;  // from the 1024-aligned shared-memory base
@@ -87,7 +92,8 @@ __device__ __forceinline__ float silu_fast(float t) { return __fdividef(t, 1.0f 
 template <int MODE, int CPL, int GS, int W, int JMAX>
 __global__ void __launch_bounds__((W + 1) * 32, 1)
     k_gemv_la(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_scales,
-              const __grid_constant__ CUtensorMap tm_biases, const LaParams p) {
+              const __grid_constant__ CUtensorMap tm_biases, const __grid_constant__ CUtensorMap tm_codes3,
+              const LaParams p) {
     constexpr int kKB = 64 * CPL * kLaSlices;  // codes per stage
     constexpr int kNB = kKB / 128;      // 128-code boxes per stage
     extern __shared__ uint8_t smem_raw[];
@@ -118,7 +124,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     if (warp == W) {
         // ---------------- producer ----------------
         if (lane == 0) {
-            prefetch_tmap(&tm_packed);
+            prefetch_tmap(p.codes3 ? &tm_codes3 : &tm_packed);
             prefetch_tmap(&tm_scales);
             prefetch_tmap(&tm_biases);
             // Warm L2 with the first stages while the previous launch finishes
@@ -145,12 +151,20 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                 if (nbox > kNB) nbox = kNB;
                 const uint32_t bar = smem_u32(&full[s]);
                 const uint32_t st = stage_of(s);
-                mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * 128u * p.R +
-                                               2u * static_cast<uint32_t>(p.R) * p.gpk * 2u);
-                for (int b = 0; b < nbox; ++b)
-                    tma_load_2d(st + static_cast<uint32_t>(b) * p.box_bytes, &tm_packed, col0 + 128 * b, r0, bar, pol);
-                tma_load_2d(st + kNB * p.box_bytes, &tm_scales, kb * p.gpk, r0, bar, pol);
-                tma_load_2d(st + kNB * p.box_bytes + p.sb_bytes, &tm_biases, kb * p.gpk, r0, bar, pol);
+                if (p.codes3) {
+                    // copies of [codes3 columns][R rows][128 bytes], zero past K
+                    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(kNB) * 128u * p.R +
+                                                   2u * static_cast<uint32_t>(p.R) * p.gpk * 2u);
+                    for (int j = 0; j < kNB; j += p.codes3)
+                        tma_load_3d(st + static_cast<uint32_t>(j) * p.box_bytes, &tm_codes3, 0, r0, kb * kNB + j, bar, pol);
+                } else {
+                    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * 128u * p.R +
+                                                   2u * static_cast<uint32_t>(p.R) * p.gpk * 2u);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(st + static_cast<uint32_t>(b) * p.box_bytes, &tm_packed, col0 + 128 * b, r0, bar, pol);
+                }
+                tma_load_2d(st + p.tab_off, &tm_scales, kb * p.gpk, r0, bar, pol);
+                tma_load_2d(st + p.tab_off + p.sb_bytes, &tm_biases, kb * p.gpk, r0, bar, pol);
                 issued = kb + 1;
             }
             if (p.pre_wait >= p.num_kb) pdl_wait();
@@ -216,7 +230,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         const int s = kb % S;
         if (ok) ok = mbar_wait(smem_u32(&full[s]), (kb / S) & 1, p.status);
         const uint32_t st = stage_of(s);
-        const uint32_t sca = st + kNB * p.box_bytes;
+        const uint32_t sca = st + p.tab_off;
         const uint32_t bia = sca + p.sb_bytes;
 #pragma unroll
         for (int j = 0; j < JMAX; ++j) {
@@ -243,7 +257,9 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                         const uint32_t xa_addr = xrow + 2u * static_cast<uint32_t>(kb * kKB + 128 * b + 16 * c);
                         xa[ci] = lds128(xa_addr);
                         xb[ci] = lds128(xa_addr + 16u);
-                        const uint32_t swz = static_cast<uint32_t>(c ^ g) << 4;
+                        // the 128-byte swizzle keys on the line's index within the
+                        // 1024-byte aligned stage: column b's rows follow column b - 1's
+                        const uint32_t swz = static_cast<uint32_t>(c ^ ((b * static_cast<int>(p.box_rows) + g) & 7)) << 4;
                         wu[ci] = lds128(boxa + swz);
                         wv[ci] = lds128(boxa + 8u * 128u + swz);
                         if (!kOneGroup || ci == 0) {
@@ -303,16 +319,28 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     }
 }
 
+struct LaMaps {
+    TensorMaps3 w;        // 2-D maps: codes [R x 128 bytes], scales and biases [R x gpk]
+    CUtensorMap codes3;   // 3-D map of the codes: one box is a stage's columns
+};
+
 constexpr int kLaW = 16;        // consumer warps
 constexpr bool kLaCpl4 = false;  // 2048-code stages for short row ranges
+// Code copies: one 2-D copy per 128-code column when the ring holds all of K
+// (every stage is issued at once, and many small copies in flight land
+// sooner: decode 4096 x 4096, 6.30 us against 6.45-6.78 with 3-D copies);
+// one 3-D copy per stage when the ring is shorter than K and a CTA has at
+// most 64 rows (8192 x 28672: 4414 -> 4767 GB/s; 4096 x 14336 down
+// projection 19.0 -> 18.6 us); per-column copies again above 64 rows.
 
 template <int MODE, int CPL, int GS, int JMAX>
-cudaError_t launch_la_t(const TensorMaps3& tm, const LaParams& p, int grid, size_t smem, cudaStream_t stream) {
+cudaError_t launch_la_t(const LaMaps& tm, const LaParams& p, int grid, size_t smem, cudaStream_t stream) {
     auto kern = k_gemv_la<MODE, CPL, GS, kLaW, JMAX>;
     static std::atomic<int> configured[64];
     cudaError_t e = ensure_dynamic_smem(kern, smem, configured);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3(grid), dim3((kLaW + 1) * 32), smem, stream, tm.packed, tm.scales, tm.biases, p);
+    e = launch_pdl(kern, dim3(grid), dim3((kLaW + 1) * 32), smem, stream, tm.w.packed, tm.w.scales, tm.w.biases,
+                   tm.codes3, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -321,7 +349,7 @@ cudaError_t launch_la_t(const TensorMaps3& tm, const LaParams& p, int grid, size
 // tiles, CPL 2 (1024) up to four tiles, CPL 1 (512) above, with 1, 2 or 4
 // items per warp; group size 128 always takes CPL >= 2 (16-byte table rows).
 template <int MODE, int CPL, int GS>
-cudaError_t launch_la_j(const TensorMaps3& tm, const LaParams& p, int jmax, int grid, size_t smem,
+cudaError_t launch_la_j(const LaMaps& tm, const LaParams& p, int jmax, int grid, size_t smem,
                         cudaStream_t stream) {
     if (jmax == 1) return launch_la_t<MODE, CPL, GS, 1>(tm, p, grid, smem, stream);
     if constexpr (CPL <= 2) {
@@ -332,7 +360,7 @@ cudaError_t launch_la_j(const TensorMaps3& tm, const LaParams& p, int jmax, int 
 }
 
 template <int MODE, int GS>
-cudaError_t launch_la_cpl(const TensorMaps3& tm, const LaParams& p, int cpl, int jmax, int grid, size_t smem,
+cudaError_t launch_la_cpl(const LaMaps& tm, const LaParams& p, int cpl, int jmax, int grid, size_t smem,
                           cudaStream_t stream) {
     if (cpl == 4) return launch_la_j<MODE, 4, GS>(tm, p, jmax, grid, smem, stream);
     if (cpl == 2) return launch_la_j<MODE, 2, GS>(tm, p, jmax, grid, smem, stream);
@@ -341,7 +369,7 @@ cudaError_t launch_la_cpl(const TensorMaps3& tm, const LaParams& p, int cpl, int
 }
 
 template <int MODE>
-cudaError_t launch_la_mode(const TensorMaps3& tm, const LaParams& p, int gs, int cpl, int jmax, int grid,
+cudaError_t launch_la_mode(const LaMaps& tm, const LaParams& p, int gs, int cpl, int jmax, int grid,
                            size_t smem, cudaStream_t stream) {
     switch (gs) {
         case 16: return launch_la_cpl<MODE, 16>(tm, p, cpl, jmax, grid, smem, stream);
@@ -357,7 +385,8 @@ bool a16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
 // Stage geometry of a weight; false if the kernel cannot take it.
 struct LaPlan {
     int cpl, R, npair, grid, num_kb, S, gpk, Kpad, pf_stages, jmax;
-    uint32_t box_bytes, sb_bytes, stage_bytes, xs_off, red_off, bar_off;
+    uint32_t box_rows, box_bytes, tab_off, sb_bytes, stage_bytes, xs_off, red_off, bar_off;
+    int codes3;
     size_t smem;
 };
 
@@ -373,24 +402,38 @@ bool plan_geometry(const WeightView& w, int mode, int R, int cpl, size_t budget,
     if (pl.gpk < 8) return false;  // a stage's table rows must be 16-byte multiples
     pl.num_kb = static_cast<int>((w.K + kb - 1) / kb);
     pl.Kpad = pl.num_kb * kb;
-    pl.box_bytes = static_cast<uint32_t>(pl.npair) * 16u * 128u;
     pl.sb_bytes = (static_cast<uint32_t>(pl.npair) * 16u * pl.gpk * 2u + 127u) / 128u * 128u;
-    pl.stage_bytes = (static_cast<uint32_t>(kb / 128) * pl.box_bytes + 2u * pl.sb_bytes + 1023u) / 1024u * 1024u;
     const uint32_t xs_bytes = static_cast<uint32_t>((mode == GEMV_PLAIN ? 2 : 4) * pl.Kpad);
     const uint32_t red_bytes = static_cast<uint32_t>(kLaSlices * pl.npair * 16 * 4);
     const size_t fixed = 1024 + xs_bytes + red_bytes + 2 * kLaMaxStages * sizeof(uint64_t);
     const int items = pl.npair * kLaSlices;
     const int j = (items + kLaW - 1) / kLaW;
     pl.jmax = j <= 1 ? 1 : (j <= 2 ? 2 : 4);
-    if (budget < fixed + static_cast<size_t>(min_stages) * pl.stage_bytes) return false;
-    int S = static_cast<int>((budget - fixed) / pl.stage_bytes);
-    if (S > kLaMaxStages) S = kLaMaxStages;
-    if (S > pl.num_kb) S = pl.num_kb;
-    pl.S = S;
-    pl.xs_off = static_cast<uint32_t>(S) * pl.stage_bytes;
-    pl.red_off = pl.xs_off + xs_bytes;
-    pl.bar_off = (pl.red_off + red_bytes + 7u) / 8u * 8u;
-    pl.smem = 1024 + pl.bar_off + 2 * kLaMaxStages * sizeof(uint64_t);
+    // The stage layout for codes3 columns per 3-D copy (0: 2-D copies).
+    // 3-D columns hold exactly R rows (K % 128 == 0); 2-D columns are padded
+    // to whole tiles.  A tile reads rows up to npair * 16 - 1 of every column,
+    // so the tables start past that.
+    auto layout = [&](int codes3) -> bool {
+        pl.codes3 = codes3;
+        pl.box_rows = codes3 ? static_cast<uint32_t>(R) : static_cast<uint32_t>(pl.npair) * 16u;
+        pl.box_bytes = pl.box_rows * 128u;
+        pl.tab_off = (static_cast<uint32_t>(kb / 128) * pl.box_bytes +
+                      (static_cast<uint32_t>(pl.npair) * 16u - pl.box_rows) * 128u + 127u) / 128u * 128u;
+        pl.stage_bytes = (pl.tab_off + 2u * pl.sb_bytes + 1023u) / 1024u * 1024u;
+        if (budget < fixed + static_cast<size_t>(min_stages) * pl.stage_bytes) return false;
+        int S = static_cast<int>((budget - fixed) / pl.stage_bytes);
+        if (S > kLaMaxStages) S = kLaMaxStages;
+        if (S > pl.num_kb) S = pl.num_kb;
+        pl.S = S;
+        pl.xs_off = static_cast<uint32_t>(S) * pl.stage_bytes;
+        pl.red_off = pl.xs_off + xs_bytes;
+        pl.bar_off = (pl.red_off + red_bytes + 7u) / 8u * 8u;
+        pl.smem = 1024 + pl.bar_off + 2 * kLaMaxStages * sizeof(uint64_t);
+        return true;
+    };
+    if (!layout(0)) return false;
+    if (pl.S < pl.num_kb && w.K % 128 == 0 && R <= 64 && !layout(kb / 128)) return false;
+    const int S = pl.S;
     // L2 prefetch of the first stages before the dependency wait, only when
     // the ring is shorter than K: otherwise every stage's copy is issued at
     // once right after the wait, and issuing the prefetches first would only
@@ -450,15 +493,23 @@ cudaError_t launch_gemv_la(const WeightView& w, int mode, const void* x, const v
     // a static weight: the ring's first stages are copied before the dependency wait
     p.pre_wait = (w.flags & MLXQ_WEIGHT_STATIC) ? pl.S : 0;
     p.pf_stages = (w.flags & MLXQ_WEIGHT_STATIC) ? 0 : pl.pf_stages;
+    p.box_rows = pl.box_rows;
     p.box_bytes = pl.box_bytes;
+    p.codes3 = pl.codes3;
+    p.tab_off = pl.tab_off;
     p.sb_bytes = pl.sb_bytes;
     p.stage_bytes = pl.stage_bytes;
     p.xs_off = pl.xs_off;
     p.red_off = pl.red_off;
     p.bar_off = pl.bar_off;
     p.status = device_status_ptr();
-    TensorMaps3 maps;
-    if (!weight_tensor_maps(w, pl.R, 128, CU_TENSOR_MAP_SWIZZLE_128B, pl.gpk, &maps)) return cudaErrorInvalidValue;
+    LaMaps maps;
+    if (!weight_tensor_maps(w, pl.R, 128, CU_TENSOR_MAP_SWIZZLE_128B, pl.gpk, &maps.w)) return cudaErrorInvalidValue;
+    std::memset(&maps.codes3, 0, sizeof(maps.codes3));
+    if (pl.codes3 && !encode_3d_chunks(&maps.codes3, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.packed, static_cast<uint64_t>(w.K),
+                                       static_cast<uint64_t>(w.N), static_cast<uint64_t>(w.K), 128,
+                                       static_cast<uint32_t>(pl.R), static_cast<uint32_t>(pl.codes3)))
+        return cudaErrorInvalidValue;
     const int gs = static_cast<int>(w.gs);
     switch (mode) {
         case GEMV_PLAIN: return launch_la_mode<GEMV_PLAIN>(maps, p, gs, pl.cpl, pl.jmax, pl.grid, pl.smem, stream);
