@@ -57,6 +57,7 @@ struct MmaParams {
     uint32_t stage_bytes;
     uint32_t x_off;         // m > 1: offset of the stage's activation boxes (1024-aligned)
     uint32_t xbox_bytes;    // m > 1: one [8 NT rows x 64 columns] BF16 box, 128-byte swizzle
+    int x3;                 // m > 1 and K % 64 == 0: the stage's boxes come as one 3-D copy
     uint32_t x_tx;          // m > 1: activation bytes per stage (0 for m == 1)
     uint32_t xs_bytes;      // activation staging (m == 1)
     unsigned int* status;
@@ -163,10 +164,15 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
                     tma_load_2d(st + static_cast<uint32_t>(b) * p.box_bytes, &tm_packed, col0 + 128 * b, r0, bar, pol);
                 tma_load_2d(st + NB * p.box_bytes, &tm_scales, kb * p.gpk, r0, bar, pol);
                 tma_load_2d(st + NB * p.box_bytes + p.sb_bytes, &tm_biases, kb * p.gpk, r0, bar, pol);
-                if constexpr (XS)  // the stage's activation columns, all 8 NT rows (zero past m and K)
-                    for (int j = 0; j < kKB / 64; ++j)
-                        tma_load_2d(st + p.x_off + static_cast<uint32_t>(j) * p.xbox_bytes, tm_x, col0 + 64 * j, 0, bar,
-                                    pol_x);
+                if constexpr (XS) {  // the stage's activation columns, all 8 NT rows (zero past m and K)
+                    if (p.x3) {  // one 3-D copy: [kKB / 64 planes][8 NT rows][64 columns]
+                        tma_load_3d(st + p.x_off, tm_x, 0, 0, col0 / 64, bar, pol_x);
+                    } else {
+                        for (int j = 0; j < kKB / 64; ++j)
+                            tma_load_2d(st + p.x_off + static_cast<uint32_t>(j) * p.xbox_bytes, tm_x, col0 + 64 * j, 0,
+                                        bar, pol_x);
+                    }
+                }
                 issued = kb + 1;
             }
             // every issued copy has landed before the CTA may exit
@@ -543,9 +549,16 @@ cudaError_t launch_stream_mma(const WeightView& w, int mode, int64_t m, const vo
     TensorMaps3 maps;
     if (!weight_tensor_maps(w, p.R, 128, CU_TENSOR_MAP_SWIZZLE_128B, p.gpk, &maps)) return cudaErrorInvalidValue;
     CUtensorMap tmx = maps.packed;  // m == 1: not read
-    if (m > 1 && !encode_2d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(w.K),
-                            static_cast<uint64_t>(m), static_cast<uint64_t>(w.K) * 2, 64,
-                            static_cast<uint32_t>(8 * nt), CU_TENSOR_MAP_SWIZZLE_128B))
+    // m > 1: the activation boxes; as 3-D planes of 64 columns (one copy per
+    // stage, the same shared-memory layout) when K % 64 == 0
+    p.x3 = (m > 1 && w.K % 64 == 0) ? 1 : 0;
+    if (p.x3 && !encode_3d_chunks(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, static_cast<uint64_t>(w.K),
+                                  static_cast<uint64_t>(m), static_cast<uint64_t>(w.K) * 2, 64,
+                                  static_cast<uint32_t>(8 * nt), static_cast<uint32_t>(kKB / 64)))
+        return cudaErrorInvalidValue;
+    if (m > 1 && !p.x3 && !encode_2d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(w.K),
+                                     static_cast<uint64_t>(m), static_cast<uint64_t>(w.K) * 2, 64,
+                                     static_cast<uint32_t>(8 * nt), CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const int grid = static_cast<int>((w.N + p.R - 1) / p.R);
     const int npair = p.R16 / 16;
