@@ -52,7 +52,10 @@ struct MmaParams {
     int R, R16;             // rows per CTA, rounded up to 16
     int num_kb, S;
     int gpk;                // scale groups per stage = 128 * NB / gs
-    uint32_t box_bytes;     // R16 * 128
+    uint32_t box_rows;      // rows of one 128-code column in shared memory (R16, or R with 3-D copies)
+    uint32_t box_bytes;     // box_rows * 128
+    int codes3;             // 1: tm_packed is a 3-D map and one copy brings a stage's NB columns
+    uint32_t tab_off;       // tables within a stage (past every row a tile reads)
     uint32_t sb_bytes;      // R16 * gpk * 2, rounded up to 128
     uint32_t stage_bytes;
     uint32_t x_off;         // m > 1: offset of the stage's activation boxes (1024-aligned)
@@ -139,7 +142,8 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
             // every load into shared memory comes after it).
             for (int kb = 0; kb < S && kb < p.num_kb; ++kb) {
                 const int col0 = kb * kKB;
-                for (int b = 0; b < NB && col0 + 128 * b < p.K; ++b) tma_prefetch_l2_2d(&tm_packed, col0 + 128 * b, r0);
+                if (!p.codes3)
+                    for (int b = 0; b < NB && col0 + 128 * b < p.K; ++b) tma_prefetch_l2_2d(&tm_packed, col0 + 128 * b, r0);
                 tma_prefetch_l2_2d(&tm_scales, kb * p.gpk, r0);
                 tma_prefetch_l2_2d(&tm_biases, kb * p.gpk, r0);
             }
@@ -158,12 +162,18 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
                 if (nbox > NB) nbox = NB;
                 const uint32_t bar = smem_u32(&full[s]);
                 const uint32_t st = stage_of(s);
-                mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * 128u * p.R +
-                                               2u * static_cast<uint32_t>(p.R) * p.gpk * 2u + p.x_tx);
-                for (int b = 0; b < nbox; ++b)
-                    tma_load_2d(st + static_cast<uint32_t>(b) * p.box_bytes, &tm_packed, col0 + 128 * b, r0, bar, pol);
-                tma_load_2d(st + NB * p.box_bytes, &tm_scales, kb * p.gpk, r0, bar, pol);
-                tma_load_2d(st + NB * p.box_bytes + p.sb_bytes, &tm_biases, kb * p.gpk, r0, bar, pol);
+                if (p.codes3) {  // one copy: [NB columns][R rows][128 bytes], zero past K
+                    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(NB) * 128u * p.R +
+                                                   2u * static_cast<uint32_t>(p.R) * p.gpk * 2u + p.x_tx);
+                    tma_load_3d(st, &tm_packed, 0, r0, kb * NB, bar, pol);
+                } else {
+                    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nbox) * 128u * p.R +
+                                                   2u * static_cast<uint32_t>(p.R) * p.gpk * 2u + p.x_tx);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(st + static_cast<uint32_t>(b) * p.box_bytes, &tm_packed, col0 + 128 * b, r0, bar, pol);
+                }
+                tma_load_2d(st + p.tab_off, &tm_scales, kb * p.gpk, r0, bar, pol);
+                tma_load_2d(st + p.tab_off + p.sb_bytes, &tm_biases, kb * p.gpk, r0, bar, pol);
                 if constexpr (XS) {  // the stage's activation columns, all 8 NT rows (zero past m and K)
                     if (p.x3) {  // one 3-D copy: [kKB / 64 planes][8 NT rows][64 columns]
                         tma_load_3d(st + p.x_off, tm_x, 0, 0, col0 / 64, bar, pol_x);
@@ -240,7 +250,9 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
     for (int ci = 0; ci < 2; ++ci) {
         const int c = tq + 4 * ci;
         grp[ci] = (box * 128 + 16 * c) / p.gs;
-        swz[ci] = static_cast<uint32_t>(c ^ g) << 4;
+        // the 128-byte swizzle keys on the line's index within the 1024-byte
+        // aligned stage: column `box`'s rows follow the previous columns'
+        swz[ci] = static_cast<uint32_t>(c ^ ((box * static_cast<int>(p.box_rows) + g) & 7)) << 4;
     }
     uint32_t rowoff[PW];
     uint32_t sbo[PW];
@@ -273,7 +285,7 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
         const bool box_in = col0 < p.K;
         const uint32_t st = stage_of(s);
         const uint32_t boxa = st + static_cast<uint32_t>(box_in ? box : 0) * p.box_bytes;
-        const uint32_t sca = st + NB * p.box_bytes;
+        const uint32_t sca = st + p.tab_off;
         const uint32_t bia = sca + p.sb_bytes;
 #pragma unroll
         for (int ci = 0; ci < 2; ++ci) {
@@ -517,38 +529,60 @@ cudaError_t launch_stream_mma(const WeightView& w, int mode, int64_t m, const vo
     if (kKB % w.gs != 0 || (kKB / w.gs) % 8 != 0) return cudaErrorInvalidValue;
     p.gpk = static_cast<int>(kKB / w.gs);
     p.num_kb = static_cast<int>((w.K + kKB - 1) / kKB);
-    p.box_bytes = static_cast<uint32_t>(p.R16) * 128u;
     p.sb_bytes = (static_cast<uint32_t>(p.R16) * p.gpk * 2u + 127u) / 128u * 128u;
-    p.stage_bytes = static_cast<uint32_t>(nb) * p.box_bytes + 2u * p.sb_bytes;
-    p.stage_bytes = (p.stage_bytes + 1023u) / 1024u * 1024u;  // keep every box 1024-byte aligned
-    if (m > 1) {  // the stage's activation slice: kKB / 64 boxes of [8 nt rows x 64 columns]
-        p.x_off = p.stage_bytes;
-        p.xbox_bytes = static_cast<uint32_t>(8 * nt) * 128u;
-        p.x_tx = static_cast<uint32_t>(kKB / 64) * p.xbox_bytes;
-        p.stage_bytes += p.x_tx;
-    }
     p.xs_bytes = (m == 1) ? static_cast<uint32_t>((mode == GEMV_PLAIN ? 2 : 4) * w.K + 127) / 128u * 128u : 0u;
     const uint32_t red_bytes = kWarps * static_cast<uint32_t>(m) * static_cast<uint32_t>(p.R16) * 4u;
     const size_t fixed = 1024 + p.xs_bytes + 2 * 16 * sizeof(uint64_t);
-    // one CTA per SM when the grid is one wave, else size for two per SM if
-    // that still leaves two stages
     const size_t full_budget = static_cast<size_t>(dev.max_smem_optin);
     const size_t half_budget = full_budget / 2 - 1024;
-    int S = static_cast<int>((full_budget - fixed) / p.stage_bytes);
-    if (waves > 1 && half_budget > fixed && (half_budget - fixed) / p.stage_bytes >= 2)
-        S = static_cast<int>((half_budget - fixed) / p.stage_bytes);
-    if (S > p.num_kb) S = p.num_kb;
-    if (S > 8) S = 8;
-    if (S < 1) return cudaErrorInvalidValue;
-    size_t smem = static_cast<size_t>(S) * p.stage_bytes + fixed;
-    if (static_cast<size_t>(S) * p.stage_bytes < red_bytes) smem = red_bytes + fixed;  // room for the final sum
-    if (smem > static_cast<size_t>(dev.max_smem_optin)) return cudaErrorInvalidValue;
-    p.S = S;
+    size_t smem = 0;
+    // The stage layout with 2-D copies of one column each (codes3 = 0,
+    // columns padded to whole tiles) or one 3-D copy of all NB columns
+    // (columns of exactly R rows; a tile reads rows up to R16 - 1 of every
+    // column, so the tables start past that).  One CTA per SM when the grid
+    // is one wave, else sized for two per SM if that still leaves two stages.
+    auto layout = [&](int codes3) -> bool {
+        p.codes3 = codes3;
+        p.box_rows = codes3 ? static_cast<uint32_t>(p.R) : static_cast<uint32_t>(p.R16);
+        p.box_bytes = p.box_rows * 128u;
+        p.tab_off = (static_cast<uint32_t>(nb) * p.box_bytes + (static_cast<uint32_t>(p.R16) - p.box_rows) * 128u + 127u) /
+                    128u * 128u;
+        p.stage_bytes = p.tab_off + 2u * p.sb_bytes;
+        p.stage_bytes = (p.stage_bytes + 1023u) / 1024u * 1024u;  // keep every stage 1024-byte aligned
+        p.x_off = 0;
+        p.xbox_bytes = 0;
+        p.x_tx = 0;
+        if (m > 1) {  // the stage's activation slice: kKB / 64 boxes of [8 nt rows x 64 columns]
+            p.x_off = p.stage_bytes;
+            p.xbox_bytes = static_cast<uint32_t>(8 * nt) * 128u;
+            p.x_tx = static_cast<uint32_t>(kKB / 64) * p.xbox_bytes;
+            p.stage_bytes += p.x_tx;
+        }
+        int S = static_cast<int>((full_budget - fixed) / p.stage_bytes);
+        if (waves > 1 && half_budget > fixed && (half_budget - fixed) / p.stage_bytes >= 2)
+            S = static_cast<int>((half_budget - fixed) / p.stage_bytes);
+        if (S > p.num_kb) S = p.num_kb;
+        if (S > 8) S = 8;
+        if (S < 1) return false;
+        smem = static_cast<size_t>(S) * p.stage_bytes + fixed;
+        if (static_cast<size_t>(S) * p.stage_bytes < red_bytes) smem = red_bytes + fixed;  // room for the final sum
+        if (smem > static_cast<size_t>(dev.max_smem_optin)) return false;
+        p.S = S;
+        return true;
+    };
+    if (!layout(0)) return cudaErrorInvalidValue;
+    // one copy per stage pays when the ring is shorter than K and the rows are
+    // few (the m = 1 kernel measured the same)
+    if (p.S < p.num_kb && w.K % 128 == 0 && p.R <= 64 && !layout(1)) return cudaErrorInvalidValue;
     p.status = device_status_ptr();
 
     TensorMaps3 maps;
     if (!weight_tensor_maps(w, p.R, 128, CU_TENSOR_MAP_SWIZZLE_128B, p.gpk, &maps)) return cudaErrorInvalidValue;
     CUtensorMap tmx = maps.packed;  // m == 1: not read
+    if (p.codes3 && !encode_3d_chunks(&maps.packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w.packed, static_cast<uint64_t>(w.K),
+                                      static_cast<uint64_t>(w.N), static_cast<uint64_t>(w.K), 128,
+                                      static_cast<uint32_t>(p.R), static_cast<uint32_t>(nb)))
+        return cudaErrorInvalidValue;
     // m > 1: the activation boxes; as 3-D planes of 64 columns (one copy per
     // stage, the same shared-memory layout) when K % 64 == 0
     p.x3 = (m > 1 && w.K % 64 == 0) ? 1 : 0;
