@@ -51,7 +51,9 @@ struct MmaParams {
     int N, K, G, gs, m;
     int R, R16;             // rows per CTA, rounded up to 16
     int num_kb, S;
-    int gpk;                // scale groups per stage = 128 * NB / gs
+    int gpk;                // scale groups per table box row: max(8, groups per stage)
+    int gstage;             // scale groups per stage = 128 * NB / gs
+    int tpair;              // 1: gstage < 8, one table box serves a pair of stages
     uint32_t box_rows;      // rows of one 128-code column in shared memory (R16, or R with 3-D copies)
     uint32_t box_bytes;     // box_rows * 128
     int codes3;             // 1: tm_packed is a 3-D map and one copy brings a stage's NB columns
@@ -144,8 +146,8 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
                 const int col0 = kb * kKB;
                 if (!p.codes3)
                     for (int b = 0; b < NB && col0 + 128 * b < p.K; ++b) tma_prefetch_l2_2d(&tm_packed, col0 + 128 * b, r0);
-                tma_prefetch_l2_2d(&tm_scales, kb * p.gpk, r0);
-                tma_prefetch_l2_2d(&tm_biases, kb * p.gpk, r0);
+                tma_prefetch_l2_2d(&tm_scales, (p.tpair ? (kb & ~1) : kb) * p.gstage, r0);
+                tma_prefetch_l2_2d(&tm_biases, (p.tpair ? (kb & ~1) : kb) * p.gstage, r0);
             }
             if constexpr (XS) prefetch_tmap(tm_x);
             pdl_wait();
@@ -172,8 +174,11 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
                     for (int b = 0; b < nbox; ++b)
                         tma_load_2d(st + static_cast<uint32_t>(b) * p.box_bytes, &tm_packed, col0 + 128 * b, r0, bar, pol);
                 }
-                tma_load_2d(st + p.tab_off, &tm_scales, kb * p.gpk, r0, bar, pol);
-                tma_load_2d(st + p.tab_off + p.sb_bytes, &tm_biases, kb * p.gpk, r0, bar, pol);
+                // the table box starts at the stage's first group, or at its
+                // pair's (fewer than 8 groups per stage: 16-byte boxes)
+                const int g0 = (p.tpair ? (kb & ~1) : kb) * p.gstage;
+                tma_load_2d(st + p.tab_off, &tm_scales, g0, r0, bar, pol);
+                tma_load_2d(st + p.tab_off + p.sb_bytes, &tm_biases, g0, r0, bar, pol);
                 if constexpr (XS) {  // the stage's activation columns, all 8 NT rows (zero past m and K)
                     if (p.x3) {  // one 3-D copy: [kKB / 64 planes][8 NT rows][64 columns]
                         tma_load_3d(st + p.x_off, tm_x, 0, 0, col0 / 64, bar, pol_x);
@@ -285,7 +290,8 @@ __device__ __forceinline__ void stream_mma(const CUtensorMap& tm_packed, const C
         const bool box_in = col0 < p.K;
         const uint32_t st = stage_of(s);
         const uint32_t boxa = st + static_cast<uint32_t>(box_in ? box : 0) * p.box_bytes;
-        const uint32_t sca = st + p.tab_off;
+        // tables: this stage's groups start (kb & 1) * gstage into a paired box
+        const uint32_t sca = st + p.tab_off + (p.tpair ? static_cast<uint32_t>((kb & 1) * p.gstage) * 2u : 0u);
         const uint32_t bia = sca + p.sb_bytes;
 #pragma unroll
         for (int ci = 0; ci < 2; ++ci) {
@@ -524,10 +530,16 @@ cudaError_t launch_stream_mma(const WeightView& w, int mode, int64_t m, const vo
     p.R16 = (p.R + 15) / 16 * 16;
     // boxes per stage: 8 while that keeps >= 3 stages in shared memory, else 4
     // (when the group size allows 4: a stage's scale box must span >= 8 groups)
-    const int nb = (p.R16 <= 64 || w.K <= 1024 || (512 / w.gs) % 8 != 0) ? 8 : 4;
+    // (a stage with fewer than 8 scale groups shares one 8-group table box
+    // with the next stage)
+    const int nb = (p.R16 <= 64 || w.K <= 1024) ? 8 : 4;
     const int kKB = 128 * nb;
-    if (kKB % w.gs != 0 || (kKB / w.gs) % 8 != 0) return cudaErrorInvalidValue;
-    p.gpk = static_cast<int>(kKB / w.gs);
+    if (kKB % w.gs != 0) return cudaErrorInvalidValue;
+    p.gstage = static_cast<int>(kKB / w.gs);
+    p.tpair = p.gstage < 8 ? 1 : 0;
+    if (p.tpair && (8 % p.gstage != 0 || 2 * p.gstage != 8)) return cudaErrorInvalidValue;
+    if (!p.tpair && p.gstage % 8 != 0) return cudaErrorInvalidValue;
+    p.gpk = p.tpair ? 8 : p.gstage;
     p.num_kb = static_cast<int>((w.K + kKB - 1) / kKB);
     p.sb_bytes = (static_cast<uint32_t>(p.R16) * p.gpk * 2u + 127u) / 128u * 128u;
     p.xs_bytes = (m == 1) ? static_cast<uint32_t>((mode == GEMV_PLAIN ? 2 : 4) * w.K + 127) / 128u * 128u : 0u;
