@@ -122,6 +122,7 @@ GEMV_SHAPES = [
     (4096, 4096, 64), (4096, 4096, 128), (4096, 4096, 32),
     (1000, 2048, 64), (333, 1024, 16), (17, 8192, 64),
     (2048, 14336, 64), (517, 14336, 128), (300, 28672, 64),  # 2 and 4 chunks per thread
+    (6000, 8192, 64),                   # 41 rows per CTA: one 3-D code copy per stage, ragged last CTA
     (129, 256, 32), (7, 64, 64), (1, 16, 16),
     (45, 36, 12), (10, 100, 4), (3, 40000, 64),              # generic path
     (700, 4096, 256), (90, 8192, 256),                        # fp32-pipe stream kernel
@@ -439,7 +440,9 @@ def run_gemm(W, X_bits, m, kernel=mq.MLXQ_GEMM_AUTO):
 
 
 SMALLM_SHAPES = [(512, 1024, 64), (300, 4096, 32), (256, 14336, 128), (128, 28672, 64), (77, 512, 16),
-                 (5000, 1152, 16), (2100, 2304, 32)]   # several tile groups per CTA; K not a multiple of 512
+                 (5000, 1152, 16), (2100, 2304, 32),   # several tile groups per CTA; K not a multiple of 512
+                 (10000, 2048, 128),   # > 64 rows per CTA at group size 128: a table box per pair of stages
+                 (9000, 8192, 64)]     # 31-61 rows per CTA: one 3-D code copy per stage
 
 
 @pytest.mark.parametrize("N,K,gs", SMALLM_SHAPES)
