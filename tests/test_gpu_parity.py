@@ -123,6 +123,8 @@ GEMV_SHAPES = [
     (1000, 2048, 64), (333, 1024, 16), (17, 8192, 64),
     (2048, 14336, 64), (517, 14336, 128), (300, 28672, 64),  # 2 and 4 chunks per thread
     (6000, 8192, 64),                   # 41 rows per CTA: one 3-D code copy per stage, ragged last CTA
+    (14336, 4096, 64), (10000, 2048, 32),  # 5 to 7 tiles per CTA: the 28-warp form, two items per warp
+    (12000, 1024, 16), (11111, 4096, 64),  # (6 tiles; 76 rows per CTA with a ragged last CTA)
     (129, 256, 32), (7, 64, 64), (1, 16, 16),
     (45, 36, 12), (10, 100, 4), (3, 40000, 64),              # generic path
     (700, 4096, 256), (90, 8192, 256),                        # fp32-pipe stream kernel
@@ -181,7 +183,7 @@ def test_gemv_integer_weights_are_exact():
 
 
 # ---------------------------------------------------------------- silu gate (+ resid)
-SILU_SHAPES = [(4096, 14336, 64), (256, 512, 64), (1000, 4096, 128), (77, 2048, 32),
+SILU_SHAPES = [(4096, 14336, 64), (256, 512, 64), (1000, 4096, 128), (77, 2048, 32), (14336, 2048, 64),
                (300, 28672, 64), (45, 36, 12),
                (500, 4096, 256), (64, 14336, 256)]   # group size the tensor-pipe kernel does not take
 
