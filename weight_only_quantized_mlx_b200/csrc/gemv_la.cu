@@ -87,8 +87,8 @@ __device__ __forceinline__ float silu_fast(float t) { return __fdividef(t, 1.0f 
 // W consumer warps (+ one producer warp).  A stage's work items are
 // (16-row tile, 64 * CPL-code slice) pairs, npair * 8 of them; warp w takes
 // items w, w + W, ... (at most JMAX), the same ones in every stage, so each
-// item has its own accumulators.  CPL: 16-code chunks per lane per item (1, 2
-// or 4; stages of 512 * CPL codes); GS: group size.
+// item has its own accumulators.  CPL: 16-code chunks per lane per item (1 or
+// 2; stages of 512 * CPL codes); GS: group size.
 template <int MODE, int CPL, int GS, int W, int JMAX>
 __global__ void __launch_bounds__((W + 1) * 32, 1)
     k_gemv_la(const __grid_constant__ CUtensorMap tm_packed, const __grid_constant__ CUtensorMap tm_scales,
@@ -325,7 +325,6 @@ struct LaMaps {
 };
 
 constexpr int kLaW = 16;        // consumer warps
-constexpr bool kLaCpl4 = false;  // 2048-code stages for short row ranges
 // Code copies: one 2-D copy per 128-code column when the ring holds all of K
 // (every stage is issued at once, and many small copies in flight land
 // sooner: decode 4096 x 4096, 6.30 us against 6.45-6.78 with 3-D copies);
@@ -345,9 +344,9 @@ cudaError_t launch_la_t(const LaMaps& tm, const LaParams& p, int grid, size_t sm
     return cudaGetLastError();
 }
 
-// Configurations the plan produces: CPL 4 (2048-code stages) for one or two
-// tiles, CPL 2 (1024) up to four tiles, CPL 1 (512) above, with 1, 2 or 4
-// items per warp; group size 128 always takes CPL >= 2 (16-byte table rows).
+// Configurations the plan produces: CPL 2 (1024-code stages) up to four
+// tiles, CPL 1 (512) above, with 1, 2 or 4 items per warp; group size 128
+// always takes CPL 2 (16-byte table rows).
 template <int MODE, int CPL, int GS>
 cudaError_t launch_la_j(const LaMaps& tm, const LaParams& p, int jmax, int grid, size_t smem,
                         cudaStream_t stream) {
@@ -362,7 +361,6 @@ cudaError_t launch_la_j(const LaMaps& tm, const LaParams& p, int jmax, int grid,
 template <int MODE, int GS>
 cudaError_t launch_la_cpl(const LaMaps& tm, const LaParams& p, int cpl, int jmax, int grid, size_t smem,
                           cudaStream_t stream) {
-    if (cpl == 4) return launch_la_j<MODE, 4, GS>(tm, p, jmax, grid, smem, stream);
     if (cpl == 2) return launch_la_j<MODE, 2, GS>(tm, p, jmax, grid, smem, stream);
     if constexpr (GS != 128) return launch_la_j<MODE, 1, GS>(tm, p, jmax, grid, smem, stream);
     return cudaErrorInvalidValue;
@@ -453,10 +451,10 @@ bool plan_la(const WeightView& w, int mode, LaPlan& pl) {
     const int npair = (R + 15) / 16;
     // Codes per stage: fewer, larger stages mean fewer stage synchronisations
     // and one scale/bias load for two chunks, as long as the ring stays deep
-    // enough: 2048 codes for up to two tiles when all of K fits in the ring,
-    // 1024 for up to four tiles, 512 above (group size 128 needs >= 1024).
+    // enough: 1024 codes for up to four tiles, 512 above (group size 128
+    // needs >= 1024).  (2048-code stages for one or two tiles measured no
+    // better at the decode shape.)
     const size_t budget = static_cast<size_t>(dev.max_smem_optin);
-    if (npair <= 2 && kLaCpl4 && plan_geometry(w, mode, R, 4, budget, 1, pl) && pl.S == pl.num_kb) return true;
     const int cpl = (w.gs == 128 || npair <= 4) ? 2 : 1;
     return plan_geometry(w, mode, R, cpl, budget, 1, pl);
 }
