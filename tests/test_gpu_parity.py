@@ -125,6 +125,7 @@ GEMV_SHAPES = [
     (6000, 8192, 64),                   # 41 rows per CTA: one 3-D code copy per stage, ragged last CTA
     (14336, 4096, 64), (10000, 2048, 32),  # 5 to 7 tiles per CTA: the 28-warp form, two items per warp
     (12000, 1024, 16), (11111, 4096, 64),  # (6 tiles; 76 rows per CTA with a ragged last CTA)
+    (20000, 1024, 64), (40000, 512, 32),   # above 128 rows per SM: the tile-group kernel at m = 1
     (129, 256, 32), (7, 64, 64), (1, 16, 16),
     (45, 36, 12), (10, 100, 4), (3, 40000, 64),              # generic path
     (700, 4096, 256), (90, 8192, 256),                        # fp32-pipe stream kernel

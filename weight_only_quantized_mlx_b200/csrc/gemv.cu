@@ -397,6 +397,12 @@ cudaError_t launch_gemv(const WeightView& w, int mode, const void* x, const void
                         const void* up, const void* resid, void* y, cudaStream_t stream) {
     if (w.N == 0) return cudaSuccess;
     if (gemv_la_supported(w, mode, x, gate, up)) return launch_gemv_la(w, mode, x, gate, up, resid, y, stream);
+    // Above 128 rows per SM (beyond k_gemv_la), the tile-group kernel at m = 1
+    // (plain gemv only) measured faster than the per-row-pair stream kernel:
+    // 28672x8192 3829 vs 3704 GB/s, 57344x4096 4042 vs 3379.
+    if (mode == GEMV_PLAIN && (w.N + device_info().sm_count - 1) / device_info().sm_count > 128 &&
+        smallm_supported(w, 1, x))
+        return launch_smallm(w, x, y, 1, stream);
     if (stream_mma_supported(w, mode, 1, x, gate, up))
         return launch_stream_mma(w, mode, 1, x, gate, up, resid, y, stream);
     const bool acts_aligned = (mode == GEMV_PLAIN) ? a16(x) : (a16(gate) && a16(up));
